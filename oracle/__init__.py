@@ -1,0 +1,294 @@
+"""CPU oracle for block-scaled FP4 (NVFP4 / MXFP4) quantization and the FP4 GEMM.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this package.
+It shares no code with the CUDA library (``block_scaled_fp4_04_b200``) and neither
+imports the other; the product path never falls back to it.
+
+The element-level definitions (code tables, encoders, quantizers, scale layout,
+dequantization) live in ``fp4_oracle.c`` and are loaded through ctypes.  The GEMM
+reference is the plain definition written out: the FP64 product of the dequantized
+operands, ``D_ref = A_hat @ B_hat^T``, with NumPy's matmul as the one library step.
+
+Sources: "Rubin FP4 GEMM overview" (yfxerp.com) 3.1 and 3.2 -- FP4 inputs, block
+scale factors re-applied to the FP32 accumulators; "FP4" glossary entry
+(ultralytics.com) "How FP4 works" -- E2M1 grid, block scale amax/6, MXFP4 and NVFP4;
+"MXFP4 / NVFP4 video transcript" (prism.simon-ai.net) -- NVFP4's FP32 tensor scale,
+16x16 weight blocks.
+
+Parity pins: every function here is pinned by a ``-m "not gpu"`` test in
+``tests/test_oracle_*.py`` (code enumeration, library conversions, the glossary's
+printed block-size experiment, hand-worked blocks, invariants, exact-rational brute
+force for the GEMM).  Parity unpinned: none of the functions below; the hardware's
+internal accumulation order is outside the oracle (covered by the GEMM tolerance).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+_lock = threading.Lock()
+
+NVFP4 = 0
+MXFP4 = 1
+F32 = 0
+BF16 = 1
+ERR_NONFINITE = 5
+
+
+def build(force: bool = False) -> str:
+    """Compile fp4_oracle.c into oracle/liboracle.so with gcc (no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-Wall",
+             "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _L():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            sig = {
+                "orc_e2m1_decode": (ctypes.c_double, [ctypes.c_uint8]),
+                "orc_e2m1_encode": (ctypes.c_uint8, [ctypes.c_float]),
+                "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
+                "orc_e4m3_encode": (ctypes.c_uint8, [ctypes.c_float]),
+                "orc_e8m0_decode": (ctypes.c_double, [ctypes.c_uint8]),
+                "orc_e8m0_encode": (ctypes.c_uint8, [ctypes.c_float]),
+                "orc_e2m1_encode_array": (None, [P, I64, P]),
+                "orc_e4m3_encode_array": (None, [P, I64, P]),
+                "orc_e8m0_encode_array": (None, [P, I64, P]),
+                "orc_amax": (I32, [P, I64, I32, P]),
+                "orc_global_scale": (ctypes.c_float, [ctypes.c_float]),
+                "orc_quantize_nvfp4_1d": (I32, [P, I64, I64, I32, P, P, P, P]),
+                "orc_quantize_mxfp4_1d": (I32, [P, I64, I64, I32, P, P]),
+                "orc_quantize_nvfp4_2d": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
+                "orc_scales_bytes": (I64, [I64, I64]),
+                "orc_swizzle_offset": (I64, [I64, I64, I64]),
+                "orc_swizzle_scales": (None, [P, I64, I64, P]),
+                "orc_unswizzle_scales": (None, [P, I64, I64, P]),
+                "orc_scales_bytes_grouped": (I64, [P, I32, I64]),
+                "orc_swizzle_scales_grouped": (None, [P, P, I32, I64, P]),
+                "orc_dequantize": (None, [P, P, ctypes.c_float, I64, I64, I32, P]),
+                "orc_fake_quant_fp32_scale": (None, [P, I64, I64, P]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class NonFiniteInput(ValueError):
+    """The tensor holds inf or NaN; no FP4 encoding is defined for it."""
+
+
+# ---------------------------------------------------------------- scalar codes
+def e2m1_decode(code: int) -> float:
+    return _L().orc_e2m1_decode(code)
+
+
+def e4m3_decode(code: int) -> float:
+    return _L().orc_e4m3_decode(code)
+
+
+def e8m0_decode(code: int) -> float:
+    return _L().orc_e8m0_decode(code)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    _L().orc_e2m1_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    _L().orc_e4m3_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e8m0_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    _L().orc_e8m0_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- tensors
+def _as_input(x: np.ndarray):
+    """float32 arrays pass as fp32; uint16 arrays are bf16 bit patterns."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, F32
+    if x.dtype == np.uint16:
+        return x, BF16
+    raise TypeError(f"oracle input must be float32 or uint16 (bf16 bits), got {x.dtype}")
+
+
+def amax(x: np.ndarray) -> float:
+    x, dt = _as_input(x)
+    out = np.zeros(1, np.float32)
+    if _L().orc_amax(_ptr(x), x.size, dt, _ptr(out)) != 0:
+        raise NonFiniteInput("non-finite element")
+    return float(out[0])
+
+
+def global_scale(amax_t: float) -> np.float32:
+    return np.float32(_L().orc_global_scale(amax_t))
+
+
+def quantize(x: np.ndarray, fmt: int = NVFP4, block: int = 16, g_in=None):
+    """Quantize a row-major [rows, cols] tensor.
+
+    Returns a dict with ``codes`` [rows, cols/2] uint8 (even element in the low
+    nibble), ``scales`` row-major [rows, cols/16 or /32] uint8, ``g`` (float32; 1.0
+    for MXFP4) and, for the 16x16 mode (block=256), ``codesT`` [cols, rows/2] and
+    ``scalesT`` [cols, rows/16].
+    """
+    x, dt = _as_input(x)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    rows, cols = x.shape
+    L = _L()
+    gbuf = np.zeros(1, np.float32)
+    gin = None
+    if g_in is not None:
+        gin = np.array([g_in], np.float32)
+    out = {}
+    if fmt == NVFP4 and block == 16:
+        codes = np.zeros((rows, cols // 2), np.uint8)
+        sc = np.zeros((rows, cols // 16), np.uint8)
+        rc = L.orc_quantize_nvfp4_1d(_ptr(x), rows, cols, dt, _ptr(gin) if gin is not None else None,
+                                     _ptr(codes), _ptr(sc), _ptr(gbuf))
+        out.update(codes=codes, scales=sc, g=np.float32(gbuf[0]))
+    elif fmt == MXFP4 and block == 32:
+        codes = np.zeros((rows, cols // 2), np.uint8)
+        sc = np.zeros((rows, cols // 32), np.uint8)
+        rc = L.orc_quantize_mxfp4_1d(_ptr(x), rows, cols, dt, _ptr(codes), _ptr(sc))
+        out.update(codes=codes, scales=sc, g=np.float32(1.0))
+    elif fmt == NVFP4 and block == 256:
+        codes = np.zeros((rows, cols // 2), np.uint8)
+        sc = np.zeros((rows, cols // 16), np.uint8)
+        codesT = np.zeros((cols, rows // 2), np.uint8)
+        scT = np.zeros((cols, rows // 16), np.uint8)
+        rc = L.orc_quantize_nvfp4_2d(_ptr(x), rows, cols, dt, _ptr(gin) if gin is not None else None,
+                                     _ptr(codes), _ptr(sc), _ptr(codesT), _ptr(scT), _ptr(gbuf))
+        out.update(codes=codes, scales=sc, codesT=codesT, scalesT=scT, g=np.float32(gbuf[0]))
+    else:
+        raise ValueError(f"unsupported fmt/block {fmt}/{block}")
+    if rc != 0:
+        raise NonFiniteInput("non-finite element")
+    return out
+
+
+def scales_bytes(rows: int, scols: int) -> int:
+    return int(_L().orc_scales_bytes(rows, scols))
+
+
+def swizzle_offset(r: int, c: int, scols: int) -> int:
+    return int(_L().orc_swizzle_offset(r, c, scols))
+
+
+def swizzle_scales(rm: np.ndarray) -> np.ndarray:
+    rm = np.ascontiguousarray(rm, dtype=np.uint8)
+    rows, scols = rm.shape
+    out = np.zeros(scales_bytes(rows, scols), np.uint8)
+    _L().orc_swizzle_scales(_ptr(rm), rows, scols, _ptr(out))
+    return out
+
+
+def unswizzle_scales(sw: np.ndarray, rows: int, scols: int) -> np.ndarray:
+    sw = np.ascontiguousarray(sw, dtype=np.uint8)
+    out = np.zeros((rows, scols), np.uint8)
+    _L().orc_unswizzle_scales(_ptr(sw), rows, scols, _ptr(out))
+    return out
+
+
+def scales_bytes_grouped(offsets: np.ndarray, scols: int) -> int:
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    return int(_L().orc_scales_bytes_grouped(_ptr(off), len(off) - 1, scols))
+
+
+def swizzle_scales_grouped(rm: np.ndarray, offsets: np.ndarray) -> np.ndarray:
+    rm = np.ascontiguousarray(rm, dtype=np.uint8)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    scols = rm.shape[1]
+    out = np.zeros(scales_bytes_grouped(off, scols), np.uint8)
+    _L().orc_swizzle_scales_grouped(_ptr(rm), _ptr(off), len(off) - 1, scols, _ptr(out))
+    return out
+
+
+def dequantize(codes: np.ndarray, scales_rm: np.ndarray, g: float, fmt: int = NVFP4) -> np.ndarray:
+    """x_hat = E2M1(code) * dec(scale) (* g for NVFP4), in float64, shape [rows, cols]."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales_rm = np.ascontiguousarray(scales_rm, dtype=np.uint8)
+    rows, half = codes.shape
+    cols = half * 2
+    out = np.zeros((rows, cols), np.float64)
+    _L().orc_dequantize(_ptr(codes), _ptr(scales_rm), float(g), rows, cols, fmt, _ptr(out))
+    return out
+
+
+def fake_quant_fp32_scale(x: np.ndarray, block: int) -> np.ndarray:
+    """The glossary experiment's procedure: unrounded FP32 block scale amax/6,
+    nearest E2M1 grid point; returns the dequantized float32 values."""
+    x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
+    out = np.zeros_like(x)
+    _L().orc_fake_quant_fp32_scale(_ptr(x), x.size, block, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- GEMM
+def gemm_reference(a_hat: np.ndarray, b_hat: np.ndarray, rows=None):
+    """FP64 definition of the block-scaled GEMM on dequantized operands.
+
+    ``D_ref[m, n] = sum_k a_hat[m, k] * b_hat[n, k]`` (A row-major [M, K], B
+    row-major [N, K], both already multiplied by their block and global scales),
+    and the tolerance base ``S[m, n] = sum_k |a_hat[m, k] * b_hat[n, k]|``.
+    ``rows`` restricts both to the listed output rows.
+    """
+    a = a_hat if rows is None else a_hat[np.asarray(rows)]
+    d = a @ b_hat.T
+    s = np.abs(a) @ np.abs(b_hat).T
+    return d, s
+
+
+def gemm_tolerance(d_ref: np.ndarray, abs_sum: np.ndarray, bf16_out: bool) -> np.ndarray:
+    """|D - D_ref| <= 1e-6 * sum_k |a_k b_k|, plus half a BF16 ulp of D_ref when the
+    output is BF16 (the larger ulp at a binade edge)."""
+    tol = 1e-6 * abs_sum
+    if bf16_out:
+        tol = tol + 0.5 * bf16_ulp(np.abs(d_ref) + tol)
+    return tol
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of BF16 values around |v| (8 significant bits); at an exact power of
+    two the larger spacing (above it) is used."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -126.0)
+    return np.ldexp(1.0, (e - 7).astype(np.int64))
