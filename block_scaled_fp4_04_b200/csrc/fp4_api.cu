@@ -1,0 +1,297 @@
+// fp4_api.cu -- the extern "C" entry points declared in include/fp4.h: argument
+// checks, workspace sizing, the per-device status word, and kernel launches.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/fp4.h"
+#include "fp4_internal.h"
+#include "fp4_ptx.cuh"
+
+namespace fp4 {
+
+// Latched device-side errors (kStatusNonFinite, kStatusTimeout); one word per device.
+__device__ unsigned g_status_word;
+
+static thread_local char g_err[256];
+
+static fp4_status fail(fp4_status s, const char* msg) {
+  snprintf(g_err, sizeof(g_err), "%s", msg);
+  return s;
+}
+
+static fp4_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_err, sizeof(g_err), "%s: %s", where, cudaGetErrorString(e));
+  return FP4_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+
+int num_sms() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// Address of this device's status word, and a check that the device is an sm_100.
+static fp4_status device_state(unsigned** status) {
+  static unsigned* addr[kMaxDevices] = {nullptr};
+  static int ok[kMaxDevices] = {0};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP4_ERR_UNSUPPORTED, "device index out of range");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ok[dev]) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return fail(FP4_ERR_UNSUPPORTED, "libfp4 is built for sm_100a (B200) only");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    addr[dev] = static_cast<unsigned*>(p);
+    ok[dev] = 1;
+  }
+  *status = addr[dev];
+  return FP4_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+const char* fp4_version(void) { return "libfp4 0.1 (sm_100a)"; }
+
+const char* fp4_last_error(void) { return g_err; }
+
+size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_fmt fmt) {
+  if (rows <= 0 || cols <= 0) return 0;
+  const int64_t blk = fmt == FP4_MXFP4 ? 32 : 16;
+  const int64_t scols = (cols + blk - 1) / blk;
+  return static_cast<size_t>(((rows + 127) / 128) * 128 * ((scols + 3) / 4) * 4);
+}
+
+size_t fp4_scales_bytes_grouped(int64_t total_rows, int num_groups, int64_t cols, fp4_fmt fmt) {
+  if (total_rows < 0 || num_groups <= 0 || cols <= 0) return 0;
+  const int64_t blk = fmt == FP4_MXFP4 ? 32 : 16;
+  const int64_t scols = (cols + blk - 1) / blk;
+  return static_cast<size_t>(((total_rows + 127) / 128 + num_groups) * 128 * ((scols + 3) / 4) * 4);
+}
+
+size_t fp4_quantize_workspace_size(void) { return kQuantWorkspaceBytes; }
+
+fp4_status fp4_amax(const void* x, int64_t n, fp4_dtype in_dtype, float* amax_out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!x || !amax_out || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (n <= 0) return fail(FP4_ERR_INVALID_ARG, "n must be positive");
+  if (in_dtype != FP4_F32 && in_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "in_dtype");
+  if (!aligned16(x) || !aligned16(workspace)) return fail(FP4_ERR_INVALID_ARG, "x and workspace must be 16-byte aligned");
+  if (workspace_bytes < kQuantWorkspaceBytes) return fail(FP4_ERR_INVALID_ARG, "workspace too small");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  cudaError_t e = launch_amax(x, n, in_dtype == FP4_BF16, static_cast<uint32_t*>(workspace), amax_out, nullptr,
+                              status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "amax launch");
+}
+
+static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
+                                  int block, uint8_t* codes, uint8_t* scales, float* gout, uint8_t* codesT,
+                                  uint8_t* scalesT, const float* gin, void* ws, size_t ws_bytes, int num_groups,
+                                  const int32_t* offsets, void* stream) {
+  if (!x || !codes || !scales) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (rows <= 0 || cols <= 0) return fail(FP4_ERR_INVALID_ARG, "rows and cols must be positive");
+  if (cols % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "cols must be a multiple of 32");
+  if (in_dtype != FP4_F32 && in_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "in_dtype");
+  if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "fmt");
+  const bool two_d = block == 256;
+  if (fmt == FP4_NVFP4 && block != 16 && block != 256) return fail(FP4_ERR_INVALID_ARG, "NVFP4 block must be 16 or 256");
+  if (fmt == FP4_MXFP4 && block != 32) return fail(FP4_ERR_INVALID_ARG, "MXFP4 block must be 32");
+  if (two_d && (!codesT || !scalesT)) return fail(FP4_ERR_INVALID_ARG, "block 256 needs codesT and scalesT");
+  if (!two_d && (codesT || scalesT)) return fail(FP4_ERR_INVALID_ARG, "codesT/scalesT only for block 256");
+  if (two_d && rows % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "block 256 needs rows % 32 == 0");
+  if (two_d && num_groups) return fail(FP4_ERR_UNSUPPORTED, "grouped 2-D quantization");
+  if (fmt == FP4_NVFP4 && !gout) return fail(FP4_ERR_INVALID_ARG, "NVFP4 needs global_out");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (codesT && !aligned16(codesT)) ||
+      (scalesT && !aligned16(scalesT)))
+    return fail(FP4_ERR_INVALID_ARG, "x, codes and scales must be 16-byte aligned");
+  if (num_groups && (num_groups > kMaxGroups || !offsets)) return fail(FP4_ERR_INVALID_ARG, "groups / offsets");
+  const bool need_amax = fmt == FP4_NVFP4 && !gin;
+  if (need_amax && (!ws || ws_bytes < kQuantWorkspaceBytes || !aligned16(ws)))
+    return fail(FP4_ERR_INVALID_ARG, "workspace too small or misaligned (fp4_quantize_workspace_size)");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bf16 = in_dtype == FP4_BF16;
+  const float* g = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (fmt == FP4_NVFP4) {
+    if (need_amax) {
+      e = launch_amax(x, rows * cols, bf16, static_cast<uint32_t*>(ws), nullptr, gout, status, st);
+      if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+      g = gout;
+    } else {
+      if (gout && gout != gin) {
+        e = cudaMemcpyAsync(gout, gin, sizeof(float), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "global scale copy");
+      }
+      g = gin;
+    }
+  } else if (gout) {
+    e = launch_set_value(gout, 1.0f, st);
+    if (e != cudaSuccess) return cuda_fail(e, "global scale write");
+  }
+  if (two_d)
+    e = launch_quantize_2d(x, rows, cols, bf16, codes, scales, codesT, scalesT, g, status, st);
+  else
+    e = launch_quantize_1d(x, rows, cols, bf16, fmt == FP4_MXFP4, codes, scales, g, offsets, num_groups, status, st);
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "quantize launch");
+}
+
+fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt, int block,
+                        uint8_t* codes_out, uint8_t* scales_out, float* global_out, uint8_t* codesT_out,
+                        uint8_t* scalesT_out, const float* global_in, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return quantize_common(x, rows, cols, in_dtype, fmt, block, codes_out, scales_out, global_out, codesT_out,
+                         scalesT_out, global_in, workspace, workspace_bytes, 0, nullptr, stream);
+}
+
+fp4_status fp4_quantize_grouped(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
+                                int num_groups, const int32_t* offsets, uint8_t* codes_out, uint8_t* scales_out,
+                                float* global_out, const float* global_in, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (num_groups <= 0) return fail(FP4_ERR_INVALID_ARG, "num_groups must be positive");
+  return quantize_common(x, rows, cols, in_dtype, fmt, fmt == FP4_MXFP4 ? 32 : 16, codes_out, scales_out,
+                         global_out, nullptr, nullptr, global_in, workspace, workspace_bytes, num_groups, offsets,
+                         stream);
+}
+
+fp4_status fp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global, int64_t rows,
+                          int64_t cols, fp4_fmt fmt, float* out, void* stream) {
+  if (!codes || !scales || !out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (rows <= 0 || cols <= 0 || cols % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "shape");
+  if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "fmt");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  cudaError_t e = launch_dequantize(codes, scales, fmt == FP4_NVFP4 ? global : nullptr, rows, cols,
+                                    fmt == FP4_MXFP4, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "dequantize launch");
+}
+
+size_t fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return gemm_workspace_bytes(M, N, K, fmt == FP4_MXFP4);
+}
+
+static fp4_status gemm_common(const GemmProblem& g, fp4_fmt fmt, fp4_dtype out_dtype, void* stream) {
+  if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "fmt");
+  if (out_dtype != FP4_F32 && out_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "out_dtype");
+  if (!g.A || !g.B || !g.sA || !g.sB || !g.D) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(FP4_ERR_INVALID_ARG, "M, N, K must be positive");
+  if (g.K % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "K must be a multiple of 32");
+  if (g.M > (1ll << 31) - 256 || g.N > (1ll << 31) - 256) return fail(FP4_ERR_UNSUPPORTED, "dimension too large");
+  if (!aligned16(g.A) || !aligned16(g.B) || !aligned16(g.sA) || !aligned16(g.sB) || !aligned16(g.D))
+    return fail(FP4_ERR_INVALID_ARG, "A, B, scales and D must be 16-byte aligned");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  const char* why = nullptr;
+  cudaError_t err = cudaSuccess;
+  const int rc = launch_gemm(g, status, static_cast<cudaStream_t>(stream), &why, &err);
+  if (rc == 1) return fail(FP4_ERR_INVALID_ARG, why);
+  if (rc == 2) return cuda_fail(err, "gemm launch");
+  return FP4_OK;
+}
+
+fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
+                    const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D, fp4_dtype out_dtype,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  GemmProblem g{};
+  g.mx = fmt == FP4_MXFP4;
+  g.A = A;
+  g.sA = sA;
+  g.gA = gA;
+  g.B = B;
+  g.sB = sB;
+  g.gB = gB;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.D = D;
+  g.out_bf16 = out_dtype == FP4_BF16;
+  g.ws = workspace;
+  g.ws_bytes = workspace_bytes;
+  return gemm_common(g, fmt, out_dtype, stream);
+}
+
+fp4_status fp4_gemm_grouped(fp4_fmt fmt, int num_groups, const int32_t* offsets, const uint8_t* A,
+                            const uint8_t* sA, const float* gA, const uint8_t* B, const uint8_t* sB,
+                            const float* gB, int64_t total_rows, int64_t N, int64_t K, void* D,
+                            fp4_dtype out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (num_groups <= 0 || num_groups > kMaxGroups || !offsets) return fail(FP4_ERR_INVALID_ARG, "groups / offsets");
+  if (N % 128 != 0) return fail(FP4_ERR_INVALID_ARG, "grouped GEMM needs N % 128 == 0");
+  if (total_rows <= 0) return fail(FP4_ERR_INVALID_ARG, "total_rows must be positive");
+  GemmProblem g{};
+  g.mx = fmt == FP4_MXFP4;
+  g.A = A;
+  g.sA = sA;
+  g.gA = gA;
+  g.B = B;
+  g.sB = sB;
+  g.gB = gB;
+  g.M = total_rows;
+  g.N = N;
+  g.K = K;
+  g.D = D;
+  g.out_bf16 = out_dtype == FP4_BF16;
+  g.ws = workspace;
+  g.ws_bytes = workspace_bytes;
+  g.num_groups = num_groups;
+  g.offsets = offsets;
+  return gemm_common(g, fmt, out_dtype, stream);
+}
+
+fp4_status fp4_get_status(void* stream) {
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  if (v & kStatusTimeout) return fail(FP4_ERR_TIMEOUT, "a device-side wait timed out");
+  if (v & kStatusNonFinite) return fail(FP4_ERR_NONFINITE, "non-finite input element");
+  return FP4_OK;
+}
+
+fp4_status fp4_debug_encode(const float* in, int64_t n, int which, uint8_t* out, void* stream) {
+  if (!in || !out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (n <= 0 || which < 0 || which > 4) return fail(FP4_ERR_INVALID_ARG, "n / which");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  cudaError_t e = launch_debug_encode(in, n, which, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "debug encode launch");
+}
+
+}  // extern "C"

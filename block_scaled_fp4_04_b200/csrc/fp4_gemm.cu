@@ -1,0 +1,725 @@
+// fp4_gemm.cu -- block-scaled FP4 GEMM on the sm_100a tensor cores (tcgen05).
+//
+// Computes D = gA * gB * (A_hat . B_hat^T) where A_hat / B_hat are E2M1 codes times
+// their block scales ("Rubin FP4 GEMM overview", yfxerp.com, 3.1: the block scale
+// factors are re-applied on the FP32 accumulators; 3.2: global -> shared -> tensor core
+// -> FP32 accumulators -> epilogue; 4.2: the global scale product is fused into the
+// epilogue so no extra pass over memory is needed).
+//
+// Structure (one CTA per SM, persistent; 6 warps):
+//   warp 0      TMA producer: per 256-wide K step, one 128x128-byte box of A, one
+//               BNx128-byte box of B (both 128-byte swizzled), and the matching
+//               512-byte scale-factor atoms by bulk copy, into a STAGES-deep ring.
+//   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale atoms -> TMEM, replicated
+//               to the 4 sub-partitions) and tcgen05.mma.kind::mxf4nvf4 (NVFP4,
+//               scale_vec::4X, UE4M3) or kind::mxf4 (MXFP4, scale_vec::2X, UE8M0),
+//               M=128, N=BN, K=64 each, accumulating in TMEM; commits free the ring
+//               slot and, at the end of a tile, hand the accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31), multiply by gA*gB, BF16 (RNE) or FP32 store; with
+//               ACC=2 accumulator buffers the epilogue of tile i overlaps tile i+1.
+// Schedules: whole tiles (grouped raster for L2 reuse), stream-K over (tile, K-step)
+// units with FP32 reduction in a workspace (decode shapes, where the small-M problem
+// runs with A and B swapped so the weight rows fill MMA-M), and grouped MoE tiles
+// enumerated on the device from the expert offsets.
+// No TMA multicast is used anywhere.  Every wait is bounded (fp4_ptx.cuh); on a timeout
+// the CTA latches the status word, drains its in-flight copies and MMAs, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fp4_internal.h"
+#include "fp4_ptx.cuh"
+
+namespace fp4 {
+
+enum { kModeTile = 0, kModeStreamK = 1, kModeGrouped = 2 };
+
+struct GemmArgs {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  int64_t sfa_rb_bytes;     // bytes per 128-row block of A's scales
+  int64_t sfb_rb_bytes;
+  int64_t sfb_group_bytes;  // grouped: bytes of one expert's B scales
+  int sf_atoms_k;           // scale atoms along K per row-block
+  int sfb_rbs;              // row-blocks of B (per expert)
+  const float* ga;
+  const float* gb;
+  int Mk, Nk, K, num_kb;    // kernel orientation
+  void* out;
+  int64_t ldo;
+  int out_bf16, transposed, vec_store;
+  float* ws;
+  int* counters;
+  int mode;
+  int tiles_m, tiles_n, group_m;
+  int64_t total_units;
+  int num_groups;
+  const int32_t* offsets;
+  int b_rows_per_group;
+  unsigned* status;
+};
+
+struct Work {
+  int a_row, b_row;    // TMA row coordinates of the A and B boxes
+  int out_row0;        // first output row (kernel orientation)
+  int rows_valid;      // rows of the tile that exist
+  int n0;              // first column (kernel orientation)
+  int sfa_rb;          // A scale row-block
+  int64_t sfb_off;     // byte offset of B's first scale row-block
+  int group;
+  int kb0, kb1;
+  int tile;
+};
+
+template <int BN>
+struct Sched {
+  const GemmArgs& p;
+  const int* s_mt;   // grouped: m-tile prefix per group
+  const int* s_off;  // grouped: row offsets
+  int64_t u, u_end;  // stream-K: current / end unit; tile modes: current unit
+  int64_t total;
+
+  __device__ Sched(const GemmArgs& args, const int* mt, const int* off) : p(args), s_mt(mt), s_off(off) {
+    if (p.mode == kModeStreamK) {
+      const int64_t T = p.total_units, G = gridDim.x;
+      u = T * blockIdx.x / G;
+      u_end = T * (blockIdx.x + 1) / G;
+      total = T;
+    } else if (p.mode == kModeGrouped) {
+      total = static_cast<int64_t>(s_mt[p.num_groups]) * p.tiles_n;
+      u = blockIdx.x;
+    } else {
+      total = p.total_units;
+      u = blockIdx.x;
+    }
+  }
+
+  __device__ bool next(Work& w) {
+    if (p.mode == kModeStreamK) {
+      if (u >= u_end) return false;
+      const int tile = static_cast<int>(u / p.num_kb);
+      const int kb0 = static_cast<int>(u % p.num_kb);
+      const int64_t kb1_ = static_cast<int64_t>(kb0) + (u_end - u);
+      const int kb1 = static_cast<int>(kb1_ < p.num_kb ? kb1_ : p.num_kb);
+      u += kb1 - kb0;
+      const int mt = tile / p.tiles_n, nt = tile % p.tiles_n;
+      plain(w, mt, nt);
+      w.kb0 = kb0;
+      w.kb1 = kb1;
+      w.tile = tile;
+      return true;
+    }
+    if (u >= total) return false;
+    const int64_t cur = u;
+    u += gridDim.x;
+    if (p.mode == kModeGrouped) {
+      const int E = p.num_groups;
+      int lo = 0, hi = E - 1;  // last group e with s_mt[e] * tiles_n <= cur
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (static_cast<int64_t>(s_mt[mid]) * p.tiles_n <= cur) lo = mid;
+        else hi = mid - 1;
+      }
+      const int e = lo;
+      const int mte = s_mt[e + 1] - s_mt[e];
+      const int64_t local = cur - static_cast<int64_t>(s_mt[e]) * p.tiles_n;
+      const int nt = static_cast<int>(local / mte), mt = static_cast<int>(local % mte);
+      w.a_row = s_off[e] + mt * 128;
+      w.out_row0 = w.a_row;
+      w.rows_valid = min(128, s_off[e + 1] - w.a_row);
+      w.n0 = nt * BN;
+      w.b_row = e * p.b_rows_per_group + w.n0;
+      w.sfa_rb = s_mt[e] + mt;
+      w.sfb_off = e * p.sfb_group_bytes + static_cast<int64_t>(w.n0 / 128) * p.sfb_rb_bytes;
+      w.group = e;
+      w.kb0 = 0;
+      w.kb1 = p.num_kb;
+      w.tile = static_cast<int>(cur);
+      return true;
+    }
+    // tile mode: rasterize in groups of group_m m-tiles so concurrently running CTAs
+    // share A and B tiles in L2
+    const int per_group = p.group_m * p.tiles_n;
+    const int gi = static_cast<int>(cur / per_group);
+    const int first_m = gi * p.group_m;
+    const int gsize = min(p.tiles_m - first_m, p.group_m);
+    const int r = static_cast<int>(cur % per_group);
+    plain(w, first_m + r % gsize, r / gsize);
+    w.kb0 = 0;
+    w.kb1 = p.num_kb;
+    w.tile = static_cast<int>(cur);
+    return true;
+  }
+
+  __device__ void plain(Work& w, int mt, int nt) {
+    w.a_row = mt * 128;
+    w.out_row0 = w.a_row;
+    w.rows_valid = min(128, p.Mk - w.a_row);
+    w.n0 = nt * BN;
+    w.b_row = w.n0;
+    w.sfa_rb = mt;
+    w.sfb_off = static_cast<int64_t>(w.n0 / 128) * p.sfb_rb_bytes;
+    w.group = 0;
+  }
+};
+
+template <int BN, bool MX, int ACC>
+struct Cfg {
+  static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
+  static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kSFABytes = kAtomsKT * 512;
+  static constexpr int kSFBBytes = kNRB * kAtomsKT * 512;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+  static constexpr int kReserve = 1024 /*align*/ + 1024 /*barriers*/ + 2 * (kMaxGroups + 1) * 4;
+  static constexpr int kStagesFit = (227 * 1024 - kReserve) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kReserve;
+  static constexpr int kSFACols = kAtomsKT * 4;
+  static constexpr int kSFBCols = kNRB * kAtomsKT * 4;
+  static constexpr int kSFSlot = kSFACols + kSFBCols;
+  static constexpr int kColsUsed = ACC * BN + 2 * kSFSlot;
+  static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                   : kColsUsed <= 256 ? 256 : 512;
+  static_assert(kColsUsed <= 512, "TMEM budget");
+  static_assert(kStages >= 2, "shared memory budget");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+};
+
+__device__ __forceinline__ void latch_timeout(volatile int* abort, unsigned* status) {
+  *abort = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// Stores 16 consecutive columns [col, col+16) of one output row (kernel orientation).
+__device__ __forceinline__ void store_row16(const GemmArgs& p, int row, int col, const float (&v)[16]) {
+  if (p.transposed) {
+    // kernel row = problem column, kernel column = problem row
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (col + j < p.Nk) {
+        const int64_t off = static_cast<int64_t>(col + j) * p.ldo + row;
+        if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[off] = __float2bfloat16_rn(v[j]);
+        else reinterpret_cast<float*>(p.out)[off] = v[j];
+      }
+    }
+    return;
+  }
+  const int64_t base = static_cast<int64_t>(row) * p.ldo + col;
+  if (p.vec_store && col + 16 <= p.Nk) {
+    if (p.out_bf16) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + base);
+      dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                          pack_bf16x2(v[6], v[7]));
+      dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                          pack_bf16x2(v[14], v[15]));
+    } else {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (col + j < p.Nk) {
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[base + j] = __float2bfloat16_rn(v[j]);
+      else reinterpret_cast<float*>(p.out)[base + j] = v[j];
+    }
+  }
+}
+
+template <int BN, bool MX, int ACC>
+__global__ void __launch_bounds__(192, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmArgs p) {
+  using C = Cfg<BN, MX, ACC>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* misc = smem + S * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint64_t* acc_empty = acc_full + ACC;
+  uint64_t* drain = acc_empty + ACC;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  volatile int* s_last = s_abort + 1;
+  volatile int* s_epi_fail = s_abort + 2;
+  int* s_mt = reinterpret_cast<int*>(misc + 1024);
+  int* s_off = s_mt + (kMaxGroups + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < ACC; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    *s_last = 0;
+    *s_epi_fail = 0;
+    fence_mbar_init();
+  }
+  if (p.mode == kModeGrouped && warp == 2) {
+    // m-tile prefix per group (= scale row-block prefix of the grouped A layout)
+    const int E = p.num_groups;
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int cnt = 0;
+      if (e < E) {
+        const int lo = p.offsets[e], hi = p.offsets[e + 1];
+        s_off[e] = lo;
+        cnt = (hi - lo + 127) / 128;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += t;
+      }
+      if (e < E) s_mt[e] = carry + incl - cnt;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) {
+      s_mt[E] = carry;
+      s_off[E] = p.offsets[E];
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t sf_col0 = ACC * BN;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      // decode streams the weights once (evict first) and re-reads the tiny activations
+      const uint64_t pol_a = p.transposed ? l2_policy_evict_first() : l2_policy_normal();
+      const uint64_t pol_b = p.transposed ? l2_policy_evict_last() : l2_policy_normal();
+      Sched<BN> sch(p, s_mt, s_off);
+      Work w;
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      while (ok && sch.next(w)) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort)) {
+            latch_timeout(s_abort, p.status);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * C::kStageBytes;
+          const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+          const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
+          const int rb0 = w.n0 / 128;
+          int nrb = 0;
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; ++rb) nrb += (rb0 + rb < p.sfb_rbs) ? 1 : 0;
+          const uint32_t bytes = C::kABytes + C::kBBytes + sf_bytes * (1 + nrb);
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(st, &tmA, &full[stage], kb * 128, w.a_row, pol_a);
+          tma_load_2d(st + C::kABytes, &tmB, &full[stage], kb * 128, w.b_row, pol_b);
+          const int64_t koff = static_cast<int64_t>(kb) * C::kAtomsKT * 512;
+          bulk_load(st + C::kABytes + C::kBBytes, p.sfa + w.sfa_rb * p.sfa_rb_bytes + koff, sf_bytes, &full[stage],
+                    pol_a);
+          for (int rb = 0; rb < nrb; ++rb)
+            bulk_load(st + C::kABytes + C::kBBytes + C::kSFABytes + rb * C::kAtomsKT * 512,
+                      p.sfb + w.sfb_off + rb * p.sfb_rb_bytes + koff, sf_bytes, &full[stage], pol_b);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*s_abort) {  // let every issued copy land before the CTA's shared memory goes away
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s)) {
+            volatile int no_abort = 0;
+            mbar_wait(&full[s], (issued_par >> s) & 1u, &no_abort);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      Sched<BN> sch(p, s_mt, s_off);
+      Work w;
+      int stage = 0, iter = 0;
+      uint32_t phase = 0, kb_iter = 0;
+      bool ok = true;
+      const uint32_t smem_base = smem_u32(smem);
+      while (ok && sch.next(w)) {
+        const int acc = iter % ACC;
+        const uint32_t acc_par = (iter / ACC) & 1;
+        if (!mbar_wait(&acc_empty[acc], acc_par ^ 1, s_abort)) {
+          latch_timeout(s_abort, p.status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * BN;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort)) {
+            latch_timeout(s_abort, p.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_base + stage * C::kStageBytes;
+          const uint32_t slot = kb_iter & 1;
+          const uint32_t sfa_t = tmem + sf_col0 + slot * C::kSFSlot;
+          const uint32_t sfb_t = sfa_t + C::kSFACols;
+          const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+          for (int a = 0; a < atoms; ++a)
+            tc_cp_sf_atom(sfa_t + a * 4, smem_desc_sf(st + C::kABytes + C::kBBytes + a * 512));
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; ++rb)
+            for (int a = 0; a < atoms; ++a)
+              tc_cp_sf_atom(sfb_t + (a * C::kNRB + rb) * 4,
+                            smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
+          const int krem = p.K - kb * 256;
+          const int nk = krem >= 256 ? 4 : (krem + 63) / 64;
+          const uint64_t adesc = smem_desc_sw128(st);
+          const uint64_t bdesc = smem_desc_sw128(st + C::kABytes);
+          for (int k = 0; k < nk; ++k) {
+            const uint32_t a_idx = MX ? (k >> 1) : k;
+            const uint32_t sfid = MX ? (k & 1) * 2 : 0;
+            const uint32_t idesc = mma_idesc(BN, MX, sfid, sfid);
+            const uint32_t accum = (kb > w.kb0 || k > 0) ? 1u : 0u;
+            const uint32_t ta = (sfa_t + a_idx * 4) | (sfid << 30);
+            const uint32_t tb = (sfb_t + a_idx * C::kNRB * 4) | (sfid << 30);
+            if constexpr (MX)
+              tc_mma_mxfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
+            else
+              tc_mma_nvfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
+          }
+          tc_commit(&empty[stage]);
+          ++kb_iter;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        ++iter;
+      }
+      // make sure no MMA still writes TMEM when it is freed
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int rl = q * 32 + lane;  // accumulator row (TMEM lane) of this thread
+    const float ga = p.ga ? *p.ga : 1.0f;
+    Sched<BN> sch(p, s_mt, s_off);
+    Work w;
+    int iter = 0;
+    while (sch.next(w)) {
+      const int acc = iter % ACC;
+      const uint32_t par = (iter / ACC) & 1;
+      // the four epilogue warps decide together whether to go on, so that none of them
+      // is left behind at a named barrier
+      if (lane == 0 && !mbar_wait(&acc_full[acc], par, s_abort)) {
+        latch_timeout(s_abort, p.status);
+        *s_epi_fail = 1;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*s_epi_fail) break;
+      tc_fence_after();
+      const float gb = p.gb ? p.gb[w.group] : 1.0f;
+      const float scale = ga * gb;
+      const bool row_ok = rl < w.rows_valid;
+      const int row = w.out_row0 + rl;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c, r);
+        tmem_ld_wait();
+        const int col = w.n0 + c;
+        if (!row_ok || col >= p.Nk) continue;
+        if (p.mode == kModeStreamK) {
+          float* dst = p.ws + static_cast<int64_t>(row) * p.Nk + col;
+          if ((p.Nk & 3) == 0 && col + 16 <= p.Nk) {
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+              red_add_v4(dst + j, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                         __uint_as_float(r[j + 3]));
+          } else {
+            for (int j = 0; j < 16 && col + j < p.Nk; ++j) atomicAdd(dst + j, __uint_as_float(r[j]));
+          }
+        } else {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]) * scale;
+          store_row16(p, row, col, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (p.mode == kModeStreamK) {
+        // the CTA that completes a tile's K range converts it and clears the workspace
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (warp == 2 && lane == 0) {
+          const int prev = atomicAdd(p.counters + w.tile, w.kb1 - w.kb0);
+          *s_last = (prev + (w.kb1 - w.kb0) == p.num_kb) ? 1 : 0;
+          if (*s_last) p.counters[w.tile] = 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*s_last) {
+          __threadfence();
+          if (row_ok) {
+            for (int c = 0; c < BN; c += 16) {
+              const int col = w.n0 + c;
+              if (col >= p.Nk) break;
+              float* src = p.ws + static_cast<int64_t>(row) * p.Nk + col;
+              float v[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                v[j] = (col + j < p.Nk) ? __ldcg(src + j) * scale : 0.0f;
+                if (col + j < p.Nk) __stcg(src + j, 0.0f);
+              }
+              store_row16(p, row, col, v);
+            }
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+      ++iter;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// [rows, inner_bytes] uint8 matrix, boxes of box_rows x 128 bytes, 128-byte swizzle,
+// out-of-bounds elements read as zero.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner_bytes, rows};
+  const cuuint64_t strides[1] = {inner_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+  bool swap;
+  int BN, ACC, mode;
+  int64_t Mk, Nk;
+  int tiles_m, tiles_n, num_kb;
+  int64_t units;
+  size_t ws_bytes;
+};
+
+static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped) {
+  Plan pl{};
+  pl.num_kb = static_cast<int>((K + 255) / 256);
+  if (grouped) {
+    pl.swap = false;
+    pl.BN = 128;
+    pl.ACC = 2;
+    pl.mode = kModeGrouped;
+    pl.Mk = M;
+    pl.Nk = N;
+    pl.tiles_n = static_cast<int>(N / 128);
+    pl.ws_bytes = 0;
+    return pl;
+  }
+  if (M <= 64) {  // decode: weight rows fill MMA-M, tokens map to MMA-N
+    pl.swap = true;
+    pl.Mk = N;
+    pl.Nk = M;
+    pl.BN = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+    pl.ACC = 2;
+  } else {
+    pl.swap = false;
+    pl.Mk = M;
+    pl.Nk = N;
+    pl.BN = N >= 256 ? 256 : 128;
+    pl.ACC = pl.BN == 256 ? 1 : 2;
+  }
+  pl.tiles_m = static_cast<int>((pl.Mk + 127) / 128);
+  pl.tiles_n = static_cast<int>((pl.Nk + pl.BN - 1) / pl.BN);
+  const int64_t tiles = static_cast<int64_t>(pl.tiles_m) * pl.tiles_n;
+  const int sms = num_sms();
+  if (pl.swap || (tiles < sms && pl.num_kb >= 4)) {
+    pl.mode = kModeStreamK;
+    pl.units = tiles * pl.num_kb;
+    pl.ws_bytes = static_cast<size_t>(pl.Mk * pl.Nk) * 4 + static_cast<size_t>(tiles) * 4 + 256;
+  } else {
+    pl.mode = kModeTile;
+    pl.units = tiles;
+    pl.ws_bytes = 0;
+  }
+  return pl;
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx) {
+  (void)mx;
+  return make_plan(M, N, K, 0).ws_bytes;
+}
+
+template <int BN, bool MX, int ACC>
+static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid, cudaStream_t st) {
+  using C = Cfg<BN, MX, ACC>;
+  auto kern = fp4_gemm_kernel<BN, MX, ACC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 192, C::kSmemBytes, st>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+template <bool MX>
+static cudaError_t dispatch(int BN, int ACC, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                            int grid, cudaStream_t st) {
+  switch (BN) {
+    case 16: return run<16, MX, 2>(ta, tb, a, grid, st);
+    case 32: return run<32, MX, 2>(ta, tb, a, grid, st);
+    case 64: return run<64, MX, 2>(ta, tb, a, grid, st);
+    case 128: return run<128, MX, 2>(ta, tb, a, grid, st);
+    default: return ACC == 1 ? run<256, MX, 1>(ta, tb, a, grid, st) : cudaErrorInvalidValue;
+  }
+}
+
+int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err) {
+  const int grouped = g.num_groups > 0;
+  const Plan pl = make_plan(g.M, g.N, g.K, grouped);
+  if (g.ws_bytes < pl.ws_bytes || (pl.ws_bytes && !g.ws)) {
+    *why = "workspace too small (see fp4_gemm_workspace_size)";
+    return 1;
+  }
+  const int64_t sf_cols = g.K / (g.mx ? 32 : 16);
+  const int64_t atoms_k = (sf_cols + 3) / 4;
+  GemmArgs a{};
+  const uint8_t *kA = g.A, *kB = g.B, *kSA = g.sA, *kSB = g.sB;
+  const float *kgA = g.gA, *kgB = g.gB;
+  int64_t rowsA = g.M, rowsB = g.N;
+  if (pl.swap) {
+    std::swap(kA, kB);
+    std::swap(kSA, kSB);
+    std::swap(kgA, kgB);
+    std::swap(rowsA, rowsB);
+  }
+  if (grouped) rowsB = static_cast<int64_t>(g.num_groups) * g.N;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, kA, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsA), 128) ||
+      !make_map(&tb, kB, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsB), static_cast<uint32_t>(pl.BN))) {
+    *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
+    return 1;
+  }
+  a.sfa = kSA;
+  a.sfb = kSB;
+  a.sfa_rb_bytes = atoms_k * 512;
+  a.sfb_rb_bytes = atoms_k * 512;
+  a.sf_atoms_k = static_cast<int>(atoms_k);
+  a.ga = kgA;
+  a.gb = kgB;
+  a.Mk = static_cast<int>(pl.Mk);
+  a.Nk = static_cast<int>(pl.Nk);
+  a.K = static_cast<int>(g.K);
+  a.num_kb = pl.num_kb;
+  a.out = g.D;
+  a.out_bf16 = g.out_bf16;
+  a.transposed = pl.swap ? 1 : 0;
+  a.ldo = pl.swap ? g.N : g.N;
+  const int esz = g.out_bf16 ? 2 : 4;
+  a.vec_store = ((g.N * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(g.D) & 15) == 0) ? 1 : 0;
+  a.mode = pl.mode;
+  a.tiles_m = pl.tiles_m;
+  a.tiles_n = pl.tiles_n;
+  a.group_m = 16;
+  a.total_units = pl.units;
+  a.status = status;
+  if (pl.mode == kModeStreamK) {
+    a.ws = static_cast<float*>(g.ws);
+    a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(g.ws) + static_cast<size_t>(pl.Mk * pl.Nk) * 4);
+  }
+  if (grouped) {
+    a.num_groups = g.num_groups;
+    a.offsets = g.offsets;
+    a.b_rows_per_group = static_cast<int>(g.N);
+    a.sfb_rbs = static_cast<int>((g.N + 127) / 128);
+    a.sfb_group_bytes = static_cast<int64_t>(a.sfb_rbs) * atoms_k * 512;
+  } else {
+    a.sfb_rbs = static_cast<int>((rowsB + 127) / 128);
+  }
+  int grid;
+  if (pl.mode == kModeGrouped) grid = num_sms();
+  else grid = static_cast<int>(std::min<int64_t>(pl.units, num_sms()));
+  grid = std::max(grid, 1);
+  const cudaError_t e = g.mx ? dispatch<true>(pl.BN, pl.ACC, ta, tb, a, grid, st)
+                             : dispatch<false>(pl.BN, pl.ACC, ta, tb, a, grid, st);
+  if (e != cudaSuccess) {
+    *err = e;
+    return 2;
+  }
+  return 0;
+}
+
+}  // namespace fp4

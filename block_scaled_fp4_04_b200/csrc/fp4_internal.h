@@ -1,0 +1,57 @@
+// fp4_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <algorithm>
+#include <cstdint>
+
+namespace fp4 {
+
+constexpr int kMaxGroups = 1024;      // grouped quantize / GEMM
+constexpr int kAmaxMaxBlocks = 1024;  // partial maxima held in the quantize workspace
+constexpr size_t kQuantWorkspaceBytes = (2 + kAmaxMaxBlocks) * sizeof(uint32_t);
+
+// Production E2M1 encoder: the hardware conversion (cvt.rn.satfinite.e2m1x2.f32) when
+// true, the threshold-count encoder when false.  Both are checked against the CPU
+// definition over every float32 bit pattern by the encoder test.
+#ifndef FP4_E2M1_HW
+#define FP4_E2M1_HW 1
+#endif
+constexpr bool kE2M1Hardware = FP4_E2M1_HW != 0;
+
+int num_sms();  // SM count of the current device (cached per device)
+
+cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float* amax_out, float* g_out,
+                        unsigned* status, cudaStream_t st);
+cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
+                               uint8_t* scales, const float* g, const int32_t* offsets, int num_groups,
+                               unsigned* status, cudaStream_t st);
+cudaError_t launch_quantize_2d(const void* x, int64_t rows, int64_t cols, int bf16, uint8_t* codes,
+                               uint8_t* scales, uint8_t* codesT, uint8_t* scalesT, const float* g,
+                               unsigned* status, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+                              int64_t cols, int mx, float* out, cudaStream_t st);
+cudaError_t launch_set_value(float* p, float v, cudaStream_t st);
+cudaError_t launch_debug_encode(const float* in, int64_t n, int which, uint8_t* out, cudaStream_t st);
+
+// GEMM problem as the host API sees it (see fp4.h for the meaning of each field).
+struct GemmProblem {
+  int mx;
+  const uint8_t *A, *sA, *B, *sB;
+  const float *gA, *gB;
+  int64_t M, N, K;
+  void* D;
+  int out_bf16;
+  void* ws;
+  size_t ws_bytes;
+  // grouped
+  int num_groups;            // 0: plain GEMM
+  const int32_t* offsets;
+};
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx);
+// Returns 0 on success, 1 on an unsupported shape / too-small workspace (message in
+// *why), or 2 on a CUDA error (code in *err).
+int launch_gemm(const GemmProblem& p, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err);
+
+}  // namespace fp4

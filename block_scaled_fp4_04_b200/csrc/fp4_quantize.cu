@@ -1,0 +1,553 @@
+// fp4_quantize.cu -- memory-bound kernels: tensor amax, 1-D and 16x16 block
+// quantization (NVFP4 / MXFP4), dequantization and the encoder check kernel.
+//
+// Method ("FP4" glossary entry, ultralytics.com, "How FP4 works"; "MXFP4 / NVFP4 video
+// transcript", prism.simon-ai.net, MXFP4 / NVFP4 / training-recipe passages):
+//   NVFP4: g = amax_t / (6*448) (1 if amax_t == 0); per 16 values sb = E4M3((amax_b/6)/g),
+//          codes = E2M1(x * (1 / (dec(sb) * g))).
+//   MXFP4: per 32 values sb = E8M0(amax_b / 6), codes = E2M1(x * 2^(127 - sb)).
+//   2-D:   NVFP4 with amax_b over a 16x16 patch; codes for W and W^T.
+// Every FP32 step is an explicit IEEE round-to-nearest operation (__fdiv_rn, __fmul_rn,
+// __frcp_rn) so that codes and scales are bit-identical to the CPU definition.
+//
+// Scale bytes are written straight into the 128x4-atom layout the tensor cores read:
+// entry (r, c) at ((r/128)*(Cpad/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "fp4_codes.cuh"
+#include "fp4_internal.h"
+#include "fp4_ptx.cuh"
+
+namespace fp4 {
+
+// ------------------------------------------------------------------ loads
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+  static constexpr int kPerChunk = 4;  // 16-byte chunk
+  __device__ __forceinline__ static void unpack(const uint4& u, float* v) {
+    v[0] = __uint_as_float(u.x);
+    v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z);
+    v[3] = __uint_as_float(u.w);
+  }
+};
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kPerChunk = 8;
+  __device__ __forceinline__ static void unpack(const uint4& u, float* v) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+// ------------------------------------------------------------------ amax
+// Grid-stride max of |x| (as bit patterns: for non-negative floats the integer order is
+// the numeric order, and inf / NaN patterns exceed every finite one).  Each block writes
+// its partial; the last block to finish (ticket from a self-resetting atomicInc) reduces
+// them, latches non-finite input, and writes amax and / or g.
+template <typename T>
+__global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, int64_t n, uint32_t* ws,
+                                                    float* amax_out, float* g_out, unsigned* status) {
+  constexpr int EPC = Elem<T>::kPerChunk;
+  const int64_t nchunks = n / EPC;
+  const uint4* xc = reinterpret_cast<const uint4*>(x);
+  uint32_t m = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < nchunks; i += 4 * stride) {
+    uint4 u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[j] = ld_stream(xc + i + j * stride);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float v[EPC];
+      Elem<T>::unpack(u[j], v);
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) m = max(m, abs_bits(v[e]));
+    }
+  }
+  for (; i < nchunks; i += stride) {
+    float v[EPC];
+    Elem<T>::unpack(ld_stream(xc + i), v);
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) m = max(m, abs_bits(v[e]));
+  }
+  if (blockIdx.x == 0) {  // tail elements that do not fill a 16-byte chunk
+    for (int64_t t = nchunks * EPC + threadIdx.x; t < n; t += blockDim.x) {
+      float v;
+      if constexpr (sizeof(T) == 4) v = reinterpret_cast<const float*>(x)[t];
+      else v = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(x)[t]) << 16);
+      m = max(m, abs_bits(v));
+    }
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t s_m[16];
+  __shared__ bool s_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_m[warp] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t bm = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) bm = max(bm, s_m[w]);
+    volatile uint32_t* partial = ws + 2;
+    partial[blockIdx.x] = bm;
+    __threadfence();
+    const unsigned ticket = atomicInc(ws, gridDim.x - 1);  // wraps back to 0 on the last block
+    s_last = (ticket == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  uint32_t bm = 0;
+  volatile uint32_t* partial = ws + 2;
+  for (unsigned b = threadIdx.x; b < gridDim.x; b += blockDim.x) bm = max(bm, partial[b]);
+  bm = __reduce_max_sync(0xFFFFFFFFu, bm);
+  if (lane == 0) s_m[warp] = bm;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t am = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) am = max(am, s_m[w]);
+    if (am >= 0x7F800000u) atomicOr(status, kStatusNonFinite);
+    const float amax = __uint_as_float(am);
+    if (amax_out) *amax_out = amax;
+    if (g_out) *g_out = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;  // 2688 = 6 * 448
+  }
+}
+
+// ------------------------------------------------------------------ group prefix
+// Row-blocks of the (grouped) scale layout: group e owns blocks [rb[e], rb[e+1]) with
+// rb[e+1] - rb[e] = ceil(rows_e / 128).  Computed by every block into shared memory.
+__device__ void group_prefix(const int32_t* offsets, int E, int* s_rb, int* s_off) {
+  // E <= kMaxGroups; simple two-level scan by one warp
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int cnt = 0;
+      if (e < E) {
+        const int lo = offsets[e], hi = offsets[e + 1];
+        s_off[e] = lo;
+        cnt = (hi - lo + 127) / 128;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += t;
+      }
+      if (e < E) s_rb[e] = carry + incl - cnt;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) {
+      s_rb[E] = carry;
+      s_off[E] = offsets[E];
+    }
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ 1-D quantize
+struct Quant1DArgs {
+  const void* x;
+  int64_t rows, cols;
+  uint8_t* codes;
+  uint8_t* scales;
+  const float* g;          // NVFP4 global scale (device)
+  const int32_t* offsets;  // grouped rows, or null
+  int num_groups;
+  int64_t rb_upper;        // row-blocks covered by the launch (grouped: upper bound)
+  int64_t ct_count;        // column tiles = atoms along columns
+  unsigned* status;
+};
+
+// One tile = 128 rows x (4 * BLOCK) columns = exactly one 512-byte scale atom.
+// 256 threads; each thread owns one 16-byte chunk per pass; the lanes of one block
+// (BLOCK / elements-per-chunk of them, adjacent) combine their maxima by shuffles.
+template <typename T, int BLOCK, bool MX, bool HW>
+__global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
+  constexpr int EPC = Elem<T>::kPerChunk;
+  constexpr int TC = 4 * BLOCK;             // columns per tile
+  constexpr int CPR = TC / EPC;             // chunks per tile row
+  constexpr int RPP = 256 / CPR;            // rows per pass
+  constexpr int PASSES = 128 / RPP;
+  constexpr int LPB = BLOCK / EPC;          // lanes per block
+  static_assert(EPC == 4 || EPC == 8, "chunk");
+
+  __shared__ __align__(16) uint8_t s_sf[512];
+  __shared__ int s_rb[kMaxGroups + 1];
+  __shared__ int s_off[kMaxGroups + 1];
+
+  const int E = p.offsets ? p.num_groups : 1;
+  if (p.offsets) {
+    group_prefix(p.offsets, E, s_rb, s_off);
+  } else {
+    if (threadIdx.x == 0) {
+      s_rb[0] = 0;
+      s_rb[1] = static_cast<int>((p.rows + 127) / 128);
+      s_off[0] = 0;
+      s_off[1] = static_cast<int>(p.rows);
+    }
+    __syncthreads();
+  }
+  const int rb_total = s_rb[E];
+  float g = 1.0f;
+  if constexpr (!MX) g = *p.g;
+
+  const int tid = threadIdx.x;
+  const int chunk = tid % CPR;
+  const int64_t half_cols = p.cols / 2;
+  const int64_t ntiles = p.rb_upper * p.ct_count;
+  unsigned bad = 0;
+
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t rb = tile / p.ct_count;
+    const int64_t ct = tile % p.ct_count;
+    uint8_t* atom = p.scales + (rb * p.ct_count + ct) * 512;
+    if (rb >= rb_total) {  // beyond the last group's blocks: zero pad atom
+      if (tid < 32) reinterpret_cast<uint4*>(atom)[tid] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    // group of this row-block (binary search over the prefix)
+    int e = 0;
+    if (E > 1) {
+      int lo = 0, hi = E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_rb[mid] <= rb) lo = mid;
+        else hi = mid - 1;
+      }
+      e = lo;
+    }
+    const int64_t row_base = s_off[e] + (rb - s_rb[e]) * 128;
+    const int64_t row_end = s_off[e + 1];
+    const int64_t col = ct * TC + chunk * EPC;
+    const bool col_ok = col < p.cols;
+
+    uint4 u[PASSES];
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int64_t r = row_base + ps * RPP + tid / CPR;
+      if (col_ok && r < row_end)
+        u[ps] = ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + col) * sizeof(T));
+      else
+        u[ps] = make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int rl = ps * RPP + tid / CPR;  // row inside the tile
+      const int64_t r = row_base + rl;
+      float v[EPC];
+      Elem<T>::unpack(u[ps], v);
+      uint32_t m = 0;
+#pragma unroll
+      for (int i = 0; i < EPC; ++i) m = max(m, abs_bits(v[i]));
+#pragma unroll
+      for (int d = 1; d < LPB; d <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+      bad |= m >= 0x7F800000u;
+      const float amax_b = __uint_as_float(m);
+      uint32_t sb;
+      float mul;
+      if constexpr (MX) {
+        sb = e8m0_code(__fdiv_rn(amax_b, 6.0f));
+        mul = e8m0_inverse(sb);
+      } else {
+        const float t = __fdiv_rn(amax_b, 6.0f);
+        sb = e4m3_code(__fdiv_rn(t, g));
+        const float denom = __fmul_rn(e4m3_value(sb), g);
+        mul = denom == 0.0f ? 0.0f : __frcp_rn(denom);
+      }
+      float s[EPC];
+#pragma unroll
+      for (int i = 0; i < EPC; ++i) s[i] = __fmul_rn(v[i], mul);
+      const bool ok = col_ok && r < row_end;
+      if constexpr (EPC == 8) {
+        const uint32_t packed = pack8<HW>(s);
+        if (ok) *reinterpret_cast<uint32_t*>(p.codes + r * half_cols + col / 2) = packed;
+      } else {
+        const uint32_t packed = pack4<HW>(s);
+        if (ok) *reinterpret_cast<uint16_t*>(p.codes + r * half_cols + col / 2) = static_cast<uint16_t>(packed);
+      }
+      if (chunk % LPB == 0) {
+        const int bc = chunk / LPB;  // block column inside the atom (0..3)
+        s_sf[(rl & 31) * 16 + (rl >> 5) * 4 + bc] = ok ? static_cast<uint8_t>(sb) : 0;
+      }
+    }
+    __syncthreads();
+    if (tid < 32) reinterpret_cast<uint4*>(atom)[tid] = reinterpret_cast<const uint4*>(s_sf)[tid];
+    __syncthreads();
+  }
+  if (bad) atomicOr(p.status, kStatusNonFinite);
+}
+
+// ------------------------------------------------------------------ 2-D quantize
+struct Quant2DArgs {
+  const void* x;
+  int64_t rows, cols;
+  uint8_t* codes;    // [rows, cols/2]
+  uint8_t* scales;   // swizzled [rows, cols/16]
+  uint8_t* codesT;   // [cols, rows/2]
+  uint8_t* scalesT;  // swizzled [cols, rows/16]
+  const float* g;
+  unsigned* status;
+};
+
+// One CTA per 128 x 128 region of W (rows and cols beyond the tensor are zero).  The
+// region is staged in shared memory (FP32, padded rows); 64 16x16 patches give 64 scale
+// bytes; then W's codes are written row-wise and W^T's codes column-wise, and both
+// scale layouts receive two full 512-byte atoms per region.
+template <typename T, bool HW>
+__global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
+  extern __shared__ __align__(16) float s_x[];  // [128][129]
+  __shared__ uint8_t s_sb[8][8];
+  __shared__ float s_mul[8][8];
+  __shared__ __align__(16) uint8_t s_atom[2][512];
+  constexpr int LD = 129;
+  const int tid = threadIdx.x;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const float g = *p.g;
+  constexpr int EPC = Elem<T>::kPerChunk;
+  constexpr int CPR = 128 / EPC;
+  unsigned bad = 0;
+
+  // stage the region
+  for (int idx = tid; idx < 128 * CPR; idx += 256) {
+    const int rl = idx / CPR, ch = idx % CPR;
+    const int64_t r = r0 + rl, c = c0 + ch * EPC;
+    float v[EPC];
+    if (r < p.rows && c < p.cols) {
+      Elem<T>::unpack(ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + c) * sizeof(T)), v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < EPC; ++i) v[i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < EPC; ++i) s_x[rl * LD + ch * EPC + i] = v[i];
+  }
+  __syncthreads();
+  // patch amax: 4 threads per patch, 4 rows each
+  {
+    const int patch = tid >> 2, sub = tid & 3;
+    const int pr = patch >> 3, pc = patch & 7;
+    uint32_t m = 0;
+    for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 16; ++j) m = max(m, abs_bits(s_x[(pr * 16 + sub * 4 + i) * LD + pc * 16 + j]));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    bad |= m >= 0x7F800000u;
+    if (sub == 0) {
+      const float amax_b = __uint_as_float(m);
+      const float t = __fdiv_rn(amax_b, 6.0f);
+      const uint32_t sb = e4m3_code(__fdiv_rn(t, g));
+      const float denom = __fmul_rn(e4m3_value(sb), g);
+      s_sb[pr][pc] = static_cast<uint8_t>(sb);
+      s_mul[pr][pc] = denom == 0.0f ? 0.0f : __frcp_rn(denom);
+    }
+  }
+  __syncthreads();
+  // W codes: thread -> (row, 16-column block); W^T codes: thread -> (col, 16-row block)
+  for (int idx = tid; idx < 128 * 8; idx += 256) {
+    const int rl = idx >> 3, bc = idx & 7;
+    const float mul = s_mul[rl >> 4][bc];
+    float a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      a[i] = __fmul_rn(s_x[rl * LD + bc * 16 + i], mul);
+      b[i] = __fmul_rn(s_x[rl * LD + bc * 16 + 8 + i], mul);
+    }
+    const int64_t r = r0 + rl, c = c0 + bc * 16;
+    const uint2 w = make_uint2(pack8<HW>(a), pack8<HW>(b));
+    if (r < p.rows && c < p.cols) *reinterpret_cast<uint2*>(p.codes + r * (p.cols / 2) + c / 2) = w;
+  }
+  for (int idx = tid; idx < 128 * 8; idx += 256) {
+    const int cl = idx & 127, br = idx >> 7;  // consecutive threads -> consecutive columns
+    const float mul = s_mul[br][cl >> 4];
+    float a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      a[i] = __fmul_rn(s_x[(br * 16 + i) * LD + cl], mul);
+      b[i] = __fmul_rn(s_x[(br * 16 + 8 + i) * LD + cl], mul);
+    }
+    const int64_t c = c0 + cl, r = r0 + br * 16;
+    const uint2 w = make_uint2(pack8<HW>(a), pack8<HW>(b));
+    if (c < p.cols && r < p.rows) *reinterpret_cast<uint2*>(p.codesT + c * (p.rows / 2) + r / 2) = w;
+  }
+  // scale atoms.  W: rows r0..r0+127, scale columns c0/16 .. +7 -> atoms (r0/128, c0/64 + {0,1}).
+  // W^T: rows c0..c0+127, scale columns r0/16 .. +7 -> atoms (c0/128, r0/64 + {0,1}).
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int idx = tid; idx < 2 * 128 * 4; idx += 256) {
+      const int a = idx >> 9, rem = idx & 511, rl = rem >> 2, cc = rem & 3;
+      const int off = (rl & 31) * 16 + (rl >> 5) * 4 + cc;
+      const int b = a * 4 + cc;  // scale column inside the region (0..7)
+      uint8_t v;
+      if (pass == 0) v = ((r0 + rl) < p.rows && (c0 + b * 16) < p.cols) ? s_sb[rl >> 4][b] : 0;
+      else v = ((c0 + rl) < p.cols && (r0 + b * 16) < p.rows) ? s_sb[b][rl >> 4] : 0;
+      s_atom[a][off] = v;
+    }
+    __syncthreads();
+    const int64_t natoms = pass == 0 ? ((p.cols / 16) + 3) / 4 : ((p.rows / 16) + 3) / 4;
+    const int64_t rowblk = pass == 0 ? r0 / 128 : c0 / 128;
+    const int64_t first = pass == 0 ? c0 / 64 : r0 / 64;
+    uint8_t* dst = pass == 0 ? p.scales : p.scalesT;
+    if (tid < 64) {
+      const int a = tid >> 5, lane = tid & 31;
+      if (first + a < natoms)
+        reinterpret_cast<uint4*>(dst + (rowblk * natoms + first + a) * 512)[lane] =
+            reinterpret_cast<const uint4*>(s_atom[a])[lane];
+    }
+    __syncthreads();
+  }
+  if (bad) atomicOr(p.status, kStatusNonFinite);
+}
+
+// ------------------------------------------------------------------ dequantize
+__global__ void dequantize_kernel(const uint8_t* codes, const uint8_t* scales, const float* gptr, int64_t rows,
+                                  int64_t cols, int mx, float* out) {
+  const int64_t n = rows * cols;
+  const int blk = mx ? 32 : 16;
+  const int64_t scols = cols / blk, cpad = (scols + 3) / 4 * 4;
+  const float g = gptr ? *gptr : 1.0f;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / cols, k = i % cols;
+    const uint8_t byte = codes[r * (cols / 2) + k / 2];
+    const uint32_t code = (k & 1) ? (byte >> 4) : (byte & 15);
+    const int64_t c = k / blk;
+    const int64_t off = ((r / 128) * (cpad / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+    const uint32_t sb = scales[off];
+    const float s = mx ? e8m0_value(sb) : __fmul_rn(e4m3_value(sb), g);
+    out[i] = __fmul_rn(e2m1_value(code), s);
+  }
+}
+
+__global__ void debug_encode_kernel(const float* in, int64_t n, int which, uint8_t* out) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = in[i];
+    uint32_t r;
+    switch (which) {
+      case 0: {  // the production encoder of the quantize kernels
+        float a[4] = {v, 0.0f, 0.0f, 0.0f};
+        r = pack4<kE2M1Hardware>(a) & 15u;
+        break;
+      }
+      case 1: r = e4m3_code(v); break;
+      case 2: r = e8m0_code(v); break;
+      case 3: r = e2m1_code_exact(v); break;
+      default: {
+        float a[4] = {v, 0.0f, 0.0f, 0.0f};
+        r = pack4<true>(a) & 15u;
+      }
+    }
+    out[i] = static_cast<uint8_t>(r);
+  }
+}
+
+__global__ void set_value_kernel(float* p, float v) { *p = v; }
+
+// ------------------------------------------------------------------ launchers
+static int blocks_for(int64_t work, int per_sm) {
+  const int sms = num_sms();
+  int64_t b = std::min<int64_t>(work, static_cast<int64_t>(sms) * per_sm);
+  return static_cast<int>(std::max<int64_t>(b, 1));
+}
+
+cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float* amax_out, float* g_out,
+                        unsigned* status, cudaStream_t st) {
+  const int epc = bf16 ? 8 : 4;
+  const int64_t chunks = (n + epc - 1) / epc;
+  int blocks = static_cast<int>(std::min<int64_t>((chunks + 2047) / 2048, static_cast<int64_t>(num_sms()) * 4));
+  blocks = std::max(1, std::min(blocks, kAmaxMaxBlocks));
+  if (bf16)
+    amax_kernel<__nv_bfloat16><<<blocks, 512, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n, ws, amax_out,
+                                                        g_out, status);
+  else
+    amax_kernel<float><<<blocks, 512, 0, st>>>(static_cast<const float*>(x), n, ws, amax_out, g_out, status);
+  return cudaGetLastError();
+}
+
+template <typename T, int BLOCK, bool MX>
+static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
+  const int blocks = blocks_for(a.rb_upper * a.ct_count, 8);
+  quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware><<<blocks, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
+                               uint8_t* scales, const float* g, const int32_t* offsets, int num_groups,
+                               unsigned* status, cudaStream_t st) {
+  Quant1DArgs a;
+  a.x = x;
+  a.rows = rows;
+  a.cols = cols;
+  a.codes = codes;
+  a.scales = scales;
+  a.g = g;
+  a.offsets = offsets;
+  a.num_groups = num_groups;
+  a.rb_upper = (rows + 127) / 128 + (offsets ? num_groups : 0);
+  const int blk = mx ? 32 : 16;
+  a.ct_count = ((cols / blk) + 3) / 4;
+  a.status = status;
+  if (bf16) return mx ? launch_q1d_t<__nv_bfloat16, 32, true>(a, st) : launch_q1d_t<__nv_bfloat16, 16, false>(a, st);
+  return mx ? launch_q1d_t<float, 32, true>(a, st) : launch_q1d_t<float, 16, false>(a, st);
+}
+
+cudaError_t launch_quantize_2d(const void* x, int64_t rows, int64_t cols, int bf16, uint8_t* codes,
+                               uint8_t* scales, uint8_t* codesT, uint8_t* scalesT, const float* g,
+                               unsigned* status, cudaStream_t st) {
+  Quant2DArgs a{x, rows, cols, codes, scales, codesT, scalesT, g, status};
+  dim3 grid(static_cast<unsigned>((cols + 127) / 128), static_cast<unsigned>((rows + 127) / 128));
+  const size_t smem = 128 * 129 * sizeof(float);
+  cudaError_t e;
+  if (bf16) {
+    e = cudaFuncSetAttribute(quantize_2d_kernel<__nv_bfloat16, kE2M1Hardware>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    quantize_2d_kernel<__nv_bfloat16, kE2M1Hardware><<<grid, 256, smem, st>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(quantize_2d_kernel<float, kE2M1Hardware>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    quantize_2d_kernel<float, kE2M1Hardware><<<grid, 256, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+                              int64_t cols, int mx, float* out, cudaStream_t st) {
+  dequantize_kernel<<<blocks_for((rows * cols + 255) / 256, 8), 256, 0, st>>>(codes, scales, g, rows, cols, mx, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_set_value(float* p, float v, cudaStream_t st) {
+  set_value_kernel<<<1, 1, 0, st>>>(p, v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_encode(const float* in, int64_t n, int which, uint8_t* out, cudaStream_t st) {
+  debug_encode_kernel<<<blocks_for((n + 255) / 256, 16), 256, 0, st>>>(in, n, which, out);
+  return cudaGetLastError();
+}
+
+}  // namespace fp4

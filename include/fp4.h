@@ -1,0 +1,178 @@
+/*
+ * fp4.h -- C ABI of libfp4: block-scaled 4-bit floating point (NVFP4, MXFP4)
+ * quantization and the FP4 GEMM that consumes it, for NVIDIA B200 (sm_100a).
+ *
+ * Value format (all entry points): E2M1 -- 1 sign, 2 exponent (bias 1), 1 mantissa
+ * bit; the only values are 0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6, no inf, no NaN
+ * ("FP4" glossary entry, ultralytics.com, opening paragraph; "Rubin FP4 GEMM
+ * overview", yfxerp.com, section 3.1 for the bit split).
+ *
+ * Block formats ("FP4" glossary entry, "How FP4 works"; "MXFP4 / NVFP4 video
+ * transcript", prism.simon-ai.net, the MXFP4 and NVFP4 passages):
+ *   NVFP4: 16 consecutive values share one E4M3 scale byte; the tensor carries one
+ *          FP32 global scale g = amax(|x|) / (6 * 448) (g = 1 for an all-zero tensor).
+ *   MXFP4: 32 consecutive values share one E8M0 (power-of-two) scale byte; g = 1.
+ *
+ * Data layouts (shared by every entry point):
+ *   codes   row-major [rows, cols/2] bytes; element 2j of a row in the low nibble of
+ *           byte j, element 2j+1 in the high nibble ("Rubin FP4 GEMM overview" 5.2
+ *           says nibble order is an API convention; this is ours).
+ *   scales  the row-major [rows, cols/block] matrix of scale bytes stored as 128x4
+ *           atoms of 512 bytes: rows padded to a multiple of 128, scale columns to a
+ *           multiple of 4 (pad bytes are written as 0).  Entry (r, c) lives at byte
+ *             ((r/128) * (Cpad/4) + c/4) * 512 + (r%32) * 16 + ((r%128)/32) * 4 + c%4
+ *           with Cpad = ceil(cols/block, 4).  This is the layout the tensor cores read
+ *           scale factors in ("Rubin FP4 GEMM overview" 4.2: the scale layout must be
+ *           tile-loadable together with the matrix).  fp4_scales_bytes() gives the size.
+ *   grouped scales (MoE activations): each group's rows start a fresh 128-row block;
+ *           group e's first block is sum_{e'<e} ceil(rows_e'/128).
+ *   GEMM    A [M, K] and B [N, K], both K-major (the contraction dimension
+ *           contiguous), D [M, N] row-major, D = (A_hat . B_hat^T) where the hats
+ *           are the dequantized operands ("Rubin FP4 GEMM overview" 3.1, 3.2: FP4
+ *           inputs, FP32 accumulation, block scales re-applied, global scales in the
+ *           epilogue per 4.2).
+ *
+ * Ownership and streams: every pointer named *_dev or documented "device" is
+ * caller-owned device memory; the library allocates no device memory in any call.
+ * All work is enqueued on the caller's stream (cudaStream_t passed as void*; NULL is
+ * the legacy default stream); no call synchronizes the host except
+ * fp4_get_status().  Global scales stay on the device (no host round trip).
+ *
+ * Errors: argument checks happen before anything is enqueued and return
+ * FP4_ERR_INVALID_ARG / FP4_ERR_UNSUPPORTED; a failed launch returns FP4_ERR_CUDA.
+ * Errors found on the device (a non-finite input element, a bounded wait that ran
+ * out) are latched in a per-device status word that fp4_get_status() reads and
+ * clears.  Outputs of a call that latched an error are unspecified.
+ */
+#ifndef FP4_H_
+#define FP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1 } fp4_fmt;
+typedef enum { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
+typedef enum {
+  FP4_OK = 0,
+  FP4_ERR_INVALID_ARG = 1, /* null pointer, bad size or alignment, too-small workspace */
+  FP4_ERR_UNSUPPORTED = 2, /* legal but not implemented combination, or no sm_100 device */
+  FP4_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  FP4_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up (latched) */
+  FP4_ERR_NONFINITE = 5    /* an input element was inf or NaN (latched) */
+} fp4_status;
+
+/* Library version string and the last host-side error message of this thread. */
+const char* fp4_version(void);
+const char* fp4_last_error(void);
+
+/* Bytes of the swizzled scale-factor buffer for a [rows, cols] tensor in fmt
+ * (block 16 for NVFP4, 32 for MXFP4): ceil(rows,128) * ceil(cols/block, 4). */
+size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_fmt fmt);
+
+/* Upper bound of the grouped scale-factor buffer for total_rows rows split into
+ * num_groups groups: (ceil(total_rows/128) + num_groups) * 128 * Cpad. */
+size_t fp4_scales_bytes_grouped(int64_t total_rows, int num_groups, int64_t cols, fp4_fmt fmt);
+
+/* Device workspace that fp4_quantize / fp4_quantize_grouped / fp4_amax need (for
+ * the tensor-amax reduction).  It must be zero-filled before its first use; every
+ * call leaves it zero-filled again.  Calls sharing one workspace must not overlap. */
+size_t fp4_quantize_workspace_size(void);
+
+/* Tensor amax ("MXFP4 / NVFP4 video transcript", NVFP4 passage: the FP32 tensor scale
+ * covers the tensor's global range): amax_out_dev[0] = max_i |x_i| over n elements of
+ * in_dtype.  A non-finite element latches FP4_ERR_NONFINITE.  x 16-byte aligned. */
+fp4_status fp4_amax(const void* x_dev, int64_t n, fp4_dtype in_dtype, float* amax_out_dev,
+                    void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Block-scaled quantization of a row-major [rows, cols] tensor ("FP4" glossary entry,
+ * "How FP4 works": the block scale maps the block's largest magnitude to 6; values
+ * round to the nearest E2M1 grid point, ties to the even mantissa; packed two per byte).
+ *   fmt/block: (FP4_NVFP4, 16) 1-D blocks along cols; (FP4_MXFP4, 32) 1-D blocks;
+ *              (FP4_NVFP4, 256) 16x16 2-D blocks for weights ("MXFP4 / NVFP4 video
+ *              transcript", training-recipe passage: W and W^T share one quantization).
+ *   codes_out_dev  [rows, cols/2]; scales_out_dev fp4_scales_bytes(rows, cols, fmt).
+ *   global_out_dev 1 float: g (NVFP4) or 1.0 (MXFP4).  May be NULL for MXFP4.
+ *   codesT_out_dev / scalesT_out_dev: block 256 only -- W^T's codes [cols, rows/2] and
+ *              scales fp4_scales_bytes(cols, rows, NVFP4); NULL otherwise.
+ *   global_in_dev: NULL -> compute amax and g on the device (two passes over x);
+ *              else the caller's g (one pass; e.g. a calibrated scale).
+ * Requires cols % 32 == 0, rows >= 1; block 256 also rows % 32 == 0; x, codes and
+ * scales 16-byte aligned.  NVFP4 block scale: sb = E4M3_rn_sat((amax_b / 6) / g);
+ * elements x * (1 / (dec(sb) * g)) in FP32.  MXFP4: sb = E8M0 nearest power of two of
+ * amax_b / 6 (a midpoint goes up); elements x * 2^(127 - sb). */
+fp4_status fp4_quantize(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype,
+                        fp4_fmt fmt, int block, uint8_t* codes_out_dev, uint8_t* scales_out_dev,
+                        float* global_out_dev, uint8_t* codesT_out_dev, uint8_t* scalesT_out_dev,
+                        const float* global_in_dev, void* workspace_dev, size_t workspace_bytes,
+                        void* stream);
+
+/* As fp4_quantize (1-D blocks) for MoE activations whose rows are grouped by expert:
+ * offsets_dev[num_groups + 1] (device int32, nondecreasing, offsets[0] = 0,
+ * offsets[num_groups] = rows) delimit the groups; scales are written in the grouped
+ * layout (size <= fp4_scales_bytes_grouped(rows, num_groups, cols, fmt); the bytes
+ * up to that bound are written, pads 0).  For NVFP4 one g covers all groups. */
+fp4_status fp4_quantize_grouped(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype,
+                                fp4_fmt fmt, int num_groups, const int32_t* offsets_dev,
+                                uint8_t* codes_out_dev, uint8_t* scales_out_dev,
+                                float* global_out_dev, const float* global_in_dev,
+                                void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Dequantize (debug / tests): out_dev[r, k] = E2M1(code) * dec(scale) * g as FP32, for a
+ * [rows, cols] tensor in the layouts above; global_dev may be NULL (g = 1). */
+fp4_status fp4_dequantize(const uint8_t* codes_dev, const uint8_t* scales_dev,
+                          const float* global_dev, int64_t rows, int64_t cols, fp4_fmt fmt,
+                          float* out_dev, void* stream);
+
+/* Device workspace bytes fp4_gemm needs for this shape (0 if none).  It must be
+ * zero-filled before first use; every call leaves it zero-filled again. */
+size_t fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt);
+
+/* Block-scaled FP4 GEMM on the 5th-generation tensor cores ("Rubin FP4 GEMM overview"
+ * 3.1-3.2 and 4.2): D[m, n] = gA * gB * sum_k dec(sA[m, k/blk]) dec(sB[n, k/blk])
+ *                             * e2m1(A[m, k]) * e2m1(B[n, k]), FP32 accumulation.
+ *   A_dev [M, K/2] codes, sA_dev scales (fp4_scales_bytes(M, K, fmt)), gA_dev 1 float
+ *   (NULL -> 1.0); B_dev [N, K/2], sB_dev, gB_dev likewise; D_dev [M, N] row-major,
+ *   out_dtype FP4_BF16 (round to nearest even) or FP4_F32.
+ * Requires K % 32 == 0, M, N >= 1, 16-byte aligned A, B, sA, sB and D.  Small M
+ * (decode) runs with A and B swapped on the tensor cores and a split over K, which
+ * uses the workspace. */
+fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,
+                    const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
+                    int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,
+                    void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Grouped (MoE) GEMM ("FP4" glossary entry, inference passage: MoE weights kept in
+ * MXFP4): for each group e, rows [offsets[e], offsets[e+1]) of A times expert e's
+ * weights B_dev + e*N*K/2 give the same rows of D:
+ *   D[r, n] = gA * gB[e] * sum_k ...   (as fp4_gemm).
+ *   A_dev [total_rows, K/2] with grouped scales sA_dev (fp4_quantize_grouped);
+ *   B_dev [num_groups, N, K/2], sB_dev num_groups consecutive fp4_scales_bytes(N, K)
+ *   blocks; gB_dev [num_groups] floats or NULL; offsets_dev device int32 [groups+1]
+ *   with offsets[num_groups] == total_rows.  D_dev [total_rows, N].
+ * Requires K % 32 == 0, N % 128 == 0, num_groups <= 1024. */
+fp4_status fp4_gemm_grouped(fp4_fmt fmt, int num_groups, const int32_t* offsets_dev,
+                            const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,
+                            const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
+                            int64_t total_rows, int64_t N, int64_t K, void* D_dev,
+                            fp4_dtype out_dtype, void* workspace_dev, size_t workspace_bytes,
+                            void* stream);
+
+/* Reads and clears the device status word latched by earlier calls on this device
+ * (after synchronizing `stream`).  Returns FP4_OK, FP4_ERR_NONFINITE or FP4_ERR_TIMEOUT
+ * (the first error latched), or FP4_ERR_CUDA if the synchronization failed. */
+fp4_status fp4_get_status(void* stream);
+
+/* Encoder check entry point (tests): out_dev[i] = the code the device encoders give
+ * in_dev[i] (no scaling), i < n.  which = 0: E2M1 code (sign in bit 3) from the encoder
+ * the quantize kernels use; 1: E4M3 scale byte of in_dev[i] >= 0; 2: E8M0 scale byte of
+ * in_dev[i] >= 0; 3: E2M1 by threshold counting; 4: E2M1 by the hardware conversion. */
+fp4_status fp4_debug_encode(const float* in_dev, int64_t n, int which, uint8_t* out_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4_H_ */

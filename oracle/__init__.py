@@ -49,7 +49,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-Wall",
+            ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-Wall", "-fopenmp",
              "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -85,6 +85,8 @@ def _L():
                 "orc_swizzle_scales_grouped": (None, [P, P, I32, I64, P]),
                 "orc_dequantize": (None, [P, P, ctypes.c_float, I64, I64, I32, P]),
                 "orc_fake_quant_fp32_scale": (None, [P, I64, I64, P]),
+                "orc_e2m1_count_mismatch": (I64, [ctypes.c_uint64, I64, P]),
+                "orc_num_threads": (I32, []),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -249,6 +251,17 @@ def dequantize(codes: np.ndarray, scales_rm: np.ndarray, g: float, fmt: int = NV
     out = np.zeros((rows, cols), np.float64)
     _L().orc_dequantize(_ptr(codes), _ptr(scales_rm), float(g), rows, cols, fmt, _ptr(out))
     return out
+
+
+def e2m1_count_mismatch(start_bits: int, codes: np.ndarray) -> int:
+    """Mismatches between codes[i] and the oracle's E2M1 code of float32 bit pattern
+    start_bits + i (NaN patterns skipped)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    return int(_L().orc_e2m1_count_mismatch(start_bits, codes.size, _ptr(codes)))
+
+
+def num_threads() -> int:
+    return int(_L().orc_num_threads())
 
 
 def fake_quant_fp32_scale(x: np.ndarray, block: int) -> np.ndarray:

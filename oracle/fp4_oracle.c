@@ -75,10 +75,23 @@ static float load_elem(const void* x, int64_t i, int dtype) {
 
 /* Magnitude of code c (0..7) from the bit fields: e = c >> 1, m = c & 1.
  * e == 0 is subnormal: m * 0.5; otherwise (1 + m/2) * 2^(e-1). */
-static double e2m1_magnitude(int c) {
+static double e2m1_magnitude_from_bits(int c) {
     int e = c >> 1, m = c & 1;
     if (e == 0) return 0.5 * m;
     return (1.0 + 0.5 * m) * ldexp(1.0, e - 1);
+}
+
+/* The same eight magnitudes, tabulated once (so that sweeps over many values do not
+ * recompute them). */
+static double e2m1_table[8];
+static int e2m1_table_ready = 0;
+
+static double e2m1_magnitude(int c) {
+    if (!e2m1_table_ready) {
+        for (int i = 0; i < 8; ++i) e2m1_table[i] = e2m1_magnitude_from_bits(i);
+        e2m1_table_ready = 1;
+    }
+    return e2m1_table[c];
 }
 
 double orc_e2m1_decode(uint8_t code) {
@@ -441,4 +454,31 @@ void orc_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
 
 void orc_e8m0_encode_array(const float* v, int64_t n, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = orc_e8m0_encode(v[i]);
+}
+
+/* Exhaustive-sweep helper: for the n float32 bit patterns start, start+1, ... compares
+ * codes[i] with orc_e2m1_encode of that pattern and returns the number of mismatches.
+ * NaN patterns (no E2M1 encoding is defined for them) are skipped.  Runs the
+ * independent elements on all OpenMP threads. */
+int64_t orc_e2m1_count_mismatch(uint64_t start, int64_t n, const uint8_t* codes) {
+    int64_t bad = 0;
+    (void)e2m1_magnitude(0); /* build the table before the threads start */
+#pragma omp parallel for reduction(+ : bad) schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t bits = (uint32_t)(start + (uint64_t)i);
+        float v;
+        memcpy(&v, &bits, 4);
+        if (isnan(v)) continue;
+        if (orc_e2m1_encode(v) != codes[i]) bad += 1;
+    }
+    return bad;
+}
+
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }

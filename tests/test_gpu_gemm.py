@@ -1,0 +1,192 @@
+"""FP4 GEMM (tcgen05) vs the FP64 oracle.
+
+Exact cases (power-of-two scales, sums exactly representable) must be bit-exact and
+pin tile coordinates, nibble order and the scale-factor layout; random cases must
+satisfy |D - D_ref| <= 1e-6 * sum_k |a_k b_k| (+ half a BF16 ulp for BF16 output)."""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_fp4_04_b200 as fp4
+import oracle
+import workloads
+from fp4_testutil import check_gemm, dequant_oracle, gpu_quantize, oracle_quantize, random_input
+
+pytestmark = pytest.mark.gpu
+
+
+def _gemm(a: fp4.Quantized, b: fp4.Quantized, out_dtype):
+    d = fp4.gemm(a, b, out_dtype)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_status() == fp4.OK
+    return d
+
+
+def _quantized_from_codes(codes_u4: np.ndarray, scale_byte: int, fmt: int) -> fp4.Quantized:
+    """Build an operand directly from 4-bit codes [rows, cols] and one scale byte."""
+    rows, cols = codes_u4.shape
+    packed = (codes_u4[:, 0::2] | (codes_u4[:, 1::2] << 4)).astype(np.uint8)
+    blk = 16 if fmt == fp4.NVFP4 else 32
+    sc = oracle.swizzle_scales(np.full((rows, cols // blk), scale_byte, np.uint8))
+    return fp4.Quantized(torch.from_numpy(packed).cuda(), torch.from_numpy(sc).cuda(),
+                         torch.ones(1, device="cuda"), rows, cols, fmt)
+
+
+def _hat(codes_u4, scale_val):
+    grid = np.array([oracle.e2m1_decode(c) for c in range(16)])
+    return grid[codes_u4] * scale_val
+
+
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
+@pytest.mark.parametrize("m,n,k", [(128, 128, 256), (130, 256, 512), (16, 384, 256), (1, 128, 64)])
+def test_identity_operand_bit_exact(fmt, m, n, k):
+    """A = identity (code 1.0 on the diagonal): D = B_hat^T restricted, exactly."""
+    a = np.zeros((m, k), np.uint8)
+    for i in range(min(m, k)):
+        a[i, i] = 2  # 1.0
+    rng = np.random.default_rng(m + n + k)
+    b = rng.integers(0, 16, (n, k)).astype(np.uint8)
+    one = 0x38 if fmt == fp4.NVFP4 else 127
+    d = _gemm(_quantized_from_codes(a, one, fmt), _quantized_from_codes(b, one, fmt), torch.float32)
+    ref = _hat(a, 1.0) @ _hat(b, 1.0).T
+    assert np.array_equal(d.cpu().numpy().astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
+def test_block_scale_placement_bit_exact(fmt):
+    """Every block has its own power-of-two scale: pins which scale byte applies to
+    which (row, K-block) on both operands."""
+    m, n, k = 256, 256, 512
+    blk = 16 if fmt == fp4.NVFP4 else 32
+    rng = np.random.default_rng(7)
+    ac = rng.integers(0, 16, (m, k)).astype(np.uint8)
+    bc = rng.integers(0, 16, (n, k)).astype(np.uint8)
+    # powers of two 2^-1 .. 2^1 on both sides: every product is a multiple of 2^-4 and
+    # |sum| < 36 * 4 * 512 < 2^17, so every partial sum needs at most 21 bits
+    if fmt == fp4.NVFP4:   # E4M3 exponent field 6..8, mantissa 0
+        a_sc = (rng.integers(6, 9, (m, k // blk)) << 3).astype(np.uint8)
+        b_sc = (rng.integers(6, 9, (n, k // blk)) << 3).astype(np.uint8)
+        val = lambda s: np.vectorize(oracle.e4m3_decode)(s)
+    else:
+        a_sc = rng.integers(126, 129, (m, k // blk)).astype(np.uint8)
+        b_sc = rng.integers(126, 129, (n, k // blk)).astype(np.uint8)
+        val = lambda s: np.vectorize(oracle.e8m0_decode)(s)
+
+    def mk(c, s):
+        packed = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+        return fp4.Quantized(torch.from_numpy(packed).cuda(), torch.from_numpy(oracle.swizzle_scales(s)).cuda(),
+                             torch.ones(1, device="cuda"), c.shape[0], c.shape[1], fmt)
+
+    d = _gemm(mk(ac, a_sc), mk(bc, b_sc), torch.float32)
+    grid = np.array([oracle.e2m1_decode(c) for c in range(16)])
+    ah = grid[ac] * np.repeat(val(a_sc), blk, 1)
+    bh = grid[bc] * np.repeat(val(b_sc), blk, 1)
+    ref = ah @ bh.T
+    assert np.array_equal(d.cpu().numpy().astype(np.float64), ref)
+
+
+def test_rank_one_integer_sums():
+    m, n, k = 200, 300, 1024
+    a = np.full((m, k), 2, np.uint8)                    # all 1.0
+    b = np.random.default_rng(3).integers(0, 16, (n, k)).astype(np.uint8)
+    d = _gemm(_quantized_from_codes(a, 0x38, fp4.NVFP4), _quantized_from_codes(b, 0x38, fp4.NVFP4), torch.float32)
+    ref = np.tile(_hat(b, 1.0).sum(1), (m, 1))
+    assert np.array_equal(d.cpu().numpy().astype(np.float64), ref)
+
+
+GEMM_CASES = [
+    # m, n, k, fmt, out dtype
+    (128, 128, 256, fp4.NVFP4, torch.float32),
+    (512, 512, 512, fp4.NVFP4, torch.float32),       # the small configuration (glossary-style inputs)
+    (200, 600, 1024, fp4.NVFP4, torch.bfloat16),     # ragged M and N
+    (256, 256, 96, fp4.NVFP4, torch.float32),        # K tail: half an MMA
+    (384, 768, 2880, fp4.MXFP4, torch.bfloat16),     # MoE K
+    (96, 256, 64, fp4.MXFP4, torch.float32),
+    (1, 256, 512, fp4.NVFP4, torch.bfloat16),        # M = 1 (swapped, split over K)
+    (16, 1024, 4096, fp4.NVFP4, torch.bfloat16),     # decode shape, reduced N
+    (40, 640, 2048, fp4.NVFP4, torch.float32),       # swapped with N-tile 64
+    (64, 384, 8192, fp4.MXFP4, torch.bfloat16),
+    (1024, 1024, 1024, fp4.NVFP4, torch.bfloat16),   # training sweep, smallest square
+]
+
+
+@pytest.mark.parametrize("m,n,k,fmt,out_dtype", GEMM_CASES)
+def test_gemm_random_within_tolerance(m, n, k, fmt, out_dtype):
+    blk = 16 if fmt == fp4.NVFP4 else 32
+    xa = random_input(m, k, m * 31 + k, torch.bfloat16)
+    xb = random_input(n, k, n * 17 + k + 1, torch.float32, std=0.02, outliers=False)
+    qa, qb = gpu_quantize(xa.cuda(), fmt, blk), gpu_quantize(xb.cuda(), fmt, blk)
+    d = _gemm(qa, qb, out_dtype)
+    oa, ob = oracle_quantize(xa, fmt, blk), oracle_quantize(xb, fmt, blk)
+    check_gemm(d, dequant_oracle(oa, fmt), dequant_oracle(ob, fmt), label=f"{m}x{n}x{k}")
+
+
+def test_gemm_pr1_configuration():
+    """512^3 NVFP4 with the seeded fp32 inputs (every 512th element x20), FP32 out."""
+    a, b = workloads.pr1_inputs()
+    qa, qb = gpu_quantize(a.cuda(), fp4.NVFP4, 16), gpu_quantize(b.cuda(), fp4.NVFP4, 16)
+    d = _gemm(qa, qb, torch.float32)
+    oa, ob = oracle_quantize(a, fp4.NVFP4, 16), oracle_quantize(b, fp4.NVFP4, 16)
+    check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label="pr1")
+
+
+def test_gemm_repeatable_and_workspace_clean():
+    """The split-over-K path leaves its workspace zero-filled; a second call agrees."""
+    xa = random_input(16, 2048, 5, torch.bfloat16)
+    xb = random_input(512, 2048, 6, torch.float32, std=0.02)
+    qa, qb = gpu_quantize(xa.cuda(), fp4.NVFP4, 16), gpu_quantize(xb.cuda(), fp4.NVFP4, 16)
+    ws = fp4.Workspace()
+    d1 = fp4.gemm(qa, qb, torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert not ws.buf.any()
+    d2 = fp4.gemm(qa, qb, torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    # FP32 partial sums meet in a different order: equal to within the tolerance
+    oa, ob = oracle_quantize(xa, fp4.NVFP4, 16), oracle_quantize(xb, fp4.NVFP4, 16)
+    for d in (d1, d2):
+        check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4))
+
+
+def test_grouped_gemm_moe_small():
+    """Grouped MXFP4 GEMM with an empty expert and ragged expert sizes."""
+    offsets = np.array([0, 130, 130, 300, 301, 560], np.int32)
+    E, N, K = len(offsets) - 1, 256, 2880
+    rows = int(offsets[-1])
+    xa = random_input(rows, K, 41, torch.bfloat16)
+    w = workloads.normal((E, N, K), 0.02, 42)
+    off_d = torch.from_numpy(offsets).cuda()
+    cap = fp4.fp4_scales_bytes_grouped(rows, E, K, fp4.MXFP4)
+    codes = torch.empty(rows, K // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(cap, dtype=torch.uint8, device="cuda")
+    fp4.fp4_quantize_grouped(xa.cuda(), rows, K, fp4.BF16, fp4.MXFP4, E, off_d, codes, scales, None)
+    wq = [gpu_quantize(w[e].cuda(), fp4.MXFP4, 32) for e in range(E)]
+    B = torch.stack([q.codes for q in wq])
+    sB = torch.cat([q.scales for q in wq])
+    D = torch.empty(rows, N, dtype=torch.bfloat16, device="cuda")
+    fp4.fp4_gemm_grouped(fp4.MXFP4, E, off_d, codes, scales, None, B, sB, None, rows, N, K, D, fp4.BF16)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_status() == fp4.OK
+    oa = oracle_quantize(xa, fp4.MXFP4, 32)
+    a_hat = dequant_oracle(oa, fp4.MXFP4)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        ob = oracle_quantize(w[e], fp4.MXFP4, 32)
+        check_gemm(D[lo:hi], a_hat[lo:hi], dequant_oracle(ob, fp4.MXFP4), label=f"expert {e}")
+
+
+def test_training_weight_reuse_forward_and_backward():
+    """One 16x16 quantization of W serves D = X W^T and dX = dY W (W^T operand)."""
+    s = 512
+    x, w, dy = workloads.train_inputs(s)
+    qw = gpu_quantize(w.cuda(), fp4.NVFP4, 256)
+    qx, qdy = gpu_quantize(x.cuda(), fp4.NVFP4, 16), gpu_quantize(dy.cuda(), fp4.NVFP4, 16)
+    d = _gemm(qx, qw, torch.bfloat16)
+    dx = _gemm(qdy, fp4.transposed(qw), torch.bfloat16)
+    ow = oracle_quantize(w, fp4.NVFP4, 256)
+    w_hat = oracle.dequantize(ow["codes"], ow["scales"], ow["g"])
+    wT_hat = oracle.dequantize(ow["codesT"], ow["scalesT"], ow["g"])
+    assert np.array_equal(w_hat.T, wT_hat)
+    check_gemm(d, dequant_oracle(oracle_quantize(x, fp4.NVFP4, 16), fp4.NVFP4), w_hat, label="fwd")
+    check_gemm(dx, dequant_oracle(oracle_quantize(dy, fp4.NVFP4, 16), fp4.NVFP4), wT_hat, label="bwd")
