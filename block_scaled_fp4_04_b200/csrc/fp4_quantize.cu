@@ -119,7 +119,10 @@ __global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, int6
   __threadfence();
   uint32_t bm = 0;
   volatile uint32_t* partial = ws + 2;
-  for (unsigned b = threadIdx.x; b < gridDim.x; b += blockDim.x) bm = max(bm, partial[b]);
+  for (unsigned b = threadIdx.x; b < gridDim.x; b += blockDim.x) {
+    bm = max(bm, partial[b]);
+    partial[b] = 0;  // leave the workspace zero-filled
+  }
   bm = __reduce_max_sync(0xFFFFFFFFu, bm);
   if (lane == 0) s_m[warp] = bm;
   __syncthreads();
@@ -279,6 +282,13 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       float s[EPC];
 #pragma unroll
       for (int i = 0; i < EPC; ++i) s[i] = __fmul_rn(v[i], mul);
+      if constexpr (!MX) {
+        if (isinf(mul)) {  // 1/denom overflowed (denom < 2^-128): zeros stay zeros, not NaN
+#pragma unroll
+          for (int i = 0; i < EPC; ++i)
+            if (v[i] == 0.0f) s[i] = v[i];
+        }
+      }
       const bool ok = col_ok && r < row_end;
       if constexpr (EPC == 8) {
         const uint32_t packed = pack8<HW>(s);
@@ -298,6 +308,9 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   }
   if (bad) atomicOr(p.status, kStatusNonFinite);
 }
+
+// x * (1/denom) with a zero element kept zero when the reciprocal overflowed.
+__device__ __forceinline__ float ratio(float x, float mul) { return x == 0.0f ? x : __fmul_rn(x, mul); }
 
 // ------------------------------------------------------------------ 2-D quantize
 struct Quant2DArgs {
@@ -372,8 +385,8 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
     float a[8], b[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      a[i] = __fmul_rn(s_x[rl * LD + bc * 16 + i], mul);
-      b[i] = __fmul_rn(s_x[rl * LD + bc * 16 + 8 + i], mul);
+      a[i] = ratio(s_x[rl * LD + bc * 16 + i], mul);
+      b[i] = ratio(s_x[rl * LD + bc * 16 + 8 + i], mul);
     }
     const int64_t r = r0 + rl, c = c0 + bc * 16;
     const uint2 w = make_uint2(pack8<HW>(a), pack8<HW>(b));
@@ -385,8 +398,8 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
     float a[8], b[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      a[i] = __fmul_rn(s_x[(br * 16 + i) * LD + cl], mul);
-      b[i] = __fmul_rn(s_x[(br * 16 + 8 + i) * LD + cl], mul);
+      a[i] = ratio(s_x[(br * 16 + i) * LD + cl], mul);
+      b[i] = ratio(s_x[(br * 16 + 8 + i) * LD + cl], mul);
     }
     const int64_t c = c0 + cl, r = r0 + br * 16;
     const uint2 w = make_uint2(pack8<HW>(a), pack8<HW>(b));

@@ -35,7 +35,8 @@
  *  - NVFP4 global scale g = amax_t / (6*448), or 1 when amax_t == 0.
  *  - NVFP4 block scale sb = E4M3((amax_b / 6) / g) (two FP32 divisions in that
  *    order); element ratio x * (1 / (dec(sb) * g)) in FP32 (one reciprocal per
- *    block, one multiply per element); a zero denominator gives zero codes.
+ *    block, one multiply per element); a zero denominator gives zero codes, and a
+ *    zero element gives a zero code even if the reciprocal overflowed.
  *  - Packing: two codes per byte, the even element in the low nibble.
  *  - Scale-factor layout: 128x4 atoms of 512 bytes (see orc_swizzle_scales).
  */
@@ -134,6 +135,18 @@ double orc_e4m3_decode(uint8_t code) {
     return s ? -v : v;
 }
 
+/* Values of the 127 finite non-negative E4M3 codes, tabulated once from the decoder. */
+static double e4m3_table[127];
+static int e4m3_table_ready = 0;
+
+static double e4m3_value(int c) {
+    if (!e4m3_table_ready) {
+        for (int i = 0; i < 127; ++i) e4m3_table[i] = orc_e4m3_decode((uint8_t)i);
+        e4m3_table_ready = 1;
+    }
+    return e4m3_table[c];
+}
+
 /* v >= 0 (may be +inf).  Nearest finite non-negative code; tie -> even mantissa;
  * above 448 the nearest finite code is 448 (saturation). */
 uint8_t orc_e4m3_encode(float v) {
@@ -142,7 +155,7 @@ uint8_t orc_e4m3_encode(float v) {
     double best_d = INFINITY;
     if (a >= 448.0) return 0x7E;  /* saturate; see orc_e2m1_encode */
     for (int c = 0; c <= 0x7E; ++c) {
-        double d = fabs(a - orc_e4m3_decode((uint8_t)c));
+        double d = fabs(a - e4m3_value(c));
         if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
             best = c;
             best_d = d;
@@ -162,6 +175,18 @@ double orc_e8m0_decode(uint8_t code) {
     return ldexp(1.0, (int)code - 127);
 }
 
+/* Values of the 255 finite E8M0 codes, tabulated once from the decoder. */
+static double e8m0_table[255];
+static int e8m0_table_ready = 0;
+
+static double e8m0_value(int c) {
+    if (!e8m0_table_ready) {
+        for (int i = 0; i < 255; ++i) e8m0_table[i] = orc_e8m0_decode((uint8_t)i);
+        e8m0_table_ready = 1;
+    }
+    return e8m0_table[c];
+}
+
 /* v >= 0.  Nearest power of two 2^(c-127), c in 0..254, in the linear domain; an
  * exact midpoint (1.5 * 2^e) goes to the larger power. */
 uint8_t orc_e8m0_encode(float v) {
@@ -169,7 +194,7 @@ uint8_t orc_e8m0_encode(float v) {
     int best = 0;
     double best_d = INFINITY;
     for (int c = 0; c <= 254; ++c) {
-        double d = isinf(a) ? (c == 254 ? 0.0 : INFINITY) : fabs(a - orc_e8m0_decode((uint8_t)c));
+        double d = isinf(a) ? (c == 254 ? 0.0 : INFINITY) : fabs(a - e8m0_value(c));
         if (d <= best_d) {  /* ascending c: an equal distance replaces with the larger power */
             best = c;
             best_d = d;
@@ -219,7 +244,10 @@ static uint8_t nvfp4_encode_block(const float* xs, int n, float amax_b, float g,
         return sb;
     }
     float inv = 1.0f / denom;
-    for (int i = 0; i < n; ++i) codes[i] = orc_e2m1_encode(xs[i] * inv);
+    /* A zero element encodes as a zero code even when 1/denom overflowed to inf
+     * (a denominator below 2^-128): the ratio x / denom of a zero is zero. */
+    for (int i = 0; i < n; ++i)
+        codes[i] = xs[i] == 0.0f ? (signbit(xs[i]) ? 8 : 0) : orc_e2m1_encode(xs[i] * inv);
     return sb;
 }
 
@@ -462,7 +490,7 @@ void orc_e8m0_encode_array(const float* v, int64_t n, uint8_t* out) {
  * independent elements on all OpenMP threads. */
 int64_t orc_e2m1_count_mismatch(uint64_t start, int64_t n, const uint8_t* codes) {
     int64_t bad = 0;
-    (void)e2m1_magnitude(0); /* build the table before the threads start */
+    (void)e2m1_magnitude(0); /* build the tables before the threads start */
 #pragma omp parallel for reduction(+ : bad) schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         uint32_t bits = (uint32_t)(start + (uint64_t)i);

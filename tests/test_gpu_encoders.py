@@ -79,13 +79,21 @@ def test_e4m3_encoder_vs_oracle_sample():
     assert np.array_equal(out.cpu().numpy(), oracle.e4m3_encode(v))
 
 
-def test_e8m0_encoder_vs_torch_every_non_negative_pattern():
-    for start in range(0, 0x7F800001, CHUNK):
-        n = min(CHUNK, 0x7F800000 - start)  # finite non-negative patterns
+def test_e8m0_encoder_vs_torch_every_normal_pattern():
+    """Normal floats vs torch (pinned to the oracle on normals); torch rounds values of
+    1.5 * 2^127 and up to NaN, which the encoder clamps to 2^127."""
+    for start in range(0x00800000, 0x7F800001, CHUNK):
+        n = min(CHUNK, 0x7F800000 - start)
         v, out = _encode_range(start, n, 2)
         ref = _torch_fp8(v, torch.float8_e8m0fnu)
-        ref = torch.where(ref == 255, torch.full_like(ref, 254), ref)  # torch rounds 2^127+ to NaN; we clamp
+        ref = torch.where(ref == 255, torch.full_like(ref, 254), ref)
         assert torch.equal(out, ref), f"chunk at {start:#x}"
+
+
+def test_e8m0_encoder_vs_oracle_every_subnormal_pattern():
+    """Zero and the subnormals (torch rounds these differently; the oracle decides)."""
+    v, out = _encode_range(0, 0x00800000, 2)
+    assert np.array_equal(out.cpu().numpy(), oracle.e8m0_encode(v.cpu().numpy()))
 
 
 def test_e8m0_encoder_vs_oracle_sample():
