@@ -203,8 +203,10 @@ def run_decode(args, dist: Dist, dev):
             raise RuntimeError(fp4.fp4_last_error())
 
     def gemm(i):
+        # pre-quantized weights: the GEMM may stream them while the activation quantize runs
         c, s, g = wp[i % copies]
-        rc = L.fp4_gemm(fp4.NVFP4, xcp, xsp, xgp, c, s, g, m, n, k, dp, fp4.BF16, gwp, gws_n, sp)
+        rc = L.fp4_gemm_ex(fp4.NVFP4, xcp, xsp, xgp, c, s, g, m, n, k, dp, fp4.BF16, gwp, gws_n,
+                           fp4.GEMM_WEIGHTS_READY, sp)
         if rc:
             raise RuntimeError(fp4.fp4_last_error())
 
@@ -292,7 +294,7 @@ def run_decode(args, dist: Dist, dev):
                          f"({copies * per_copy / 2**20:.0f} MiB > 126 MiB L2)",
                    "parallelism": f"replicas x{dist.world} (independent problems)"},
         "tflops": 2.0 * m * n * k * dist.world / (max_ms / K * 1e-3) / 1e12,
-        "roofline": {"bound": "hbm", "kernel": "fp4_gemm_kernel<16,nvfp4> (swapped, split over K)",
+        "roofline": {"bound": "hbm", "kernel": "fp4_gemm_kernel<16,nvfp4,2> + splitk_finalize (swapped, stream-K)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": f"{src} hbm_gbs (MEASURED_PEAKS.json)" if src == "measured" else src,
                      "algorithmic_bytes_per_launch": gb, "launch_ms": gemm_avg_ms,
@@ -300,7 +302,8 @@ def run_decode(args, dist: Dist, dev):
         "e2e": {"value": whole_job_value(step_bytes * K, dist.world, e2e_ms) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2,
                 "ms_per_step": e2e_ms / K},
-        "gpu_launches": 3 * K,
+        # per step: amax, quantize, GEMM and its split-K finalize
+        "gpu_launches": 4 * K,
         "clocks": clk,
     }
     return res

@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libfp4.so")
 NVFP4, MXFP4 = 0, 1
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = range(6)
+GEMM_WEIGHTS_READY = 1
 _STATUS_NAMES = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED", 3: "FP4_ERR_CUDA",
                  4: "FP4_ERR_TIMEOUT", 5: "FP4_ERR_NONFINITE"}
 
@@ -60,6 +61,7 @@ def lib() -> ctypes.CDLL:
                 "fp4_dequantize": (I32, [P, P, P, I64, I64, I32, P, P]),
                 "fp4_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
                 "fp4_gemm": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
+                "fp4_gemm_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_grouped": (I32, [I32, I32, P, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_get_status": (I32, [P]),
                 "fp4_debug_encode": (I32, [P, I64, I32, P, P]),
@@ -152,6 +154,12 @@ def fp4_dequantize(codes, scales, global_, rows, cols, fmt, out, stream=None):
 def fp4_gemm(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace=None, workspace_bytes=0, stream=None):
     _check(lib().fp4_gemm(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype,
                           _p(workspace), workspace_bytes, _s(stream)))
+
+
+def fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace=None, workspace_bytes=0, flags=0,
+                stream=None):
+    _check(lib().fp4_gemm_ex(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype,
+                             _p(workspace), workspace_bytes, flags, _s(stream)))
 
 
 def fp4_gemm_grouped(fmt, num_groups, offsets, A, sA, gA, B, sB, gB, total_rows, N, K, D, out_dtype,

@@ -5,7 +5,7 @@
 #include <cstdio>
 #include <mutex>
 
-#include "../../include/fp4.h"
+#include "fp4.h"
 #include "fp4_internal.h"
 #include "fp4_ptx.cuh"
 
@@ -219,9 +219,11 @@ static fp4_status gemm_common(const GemmProblem& g, fp4_fmt fmt, fp4_dtype out_d
   return FP4_OK;
 }
 
-fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
-                    const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D, fp4_dtype out_dtype,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
+                       const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D,
+                       fp4_dtype out_dtype, void* workspace, size_t workspace_bytes, unsigned flags,
+                       void* stream) {
+  if (flags & ~static_cast<unsigned>(FP4_GEMM_WEIGHTS_READY)) return fail(FP4_ERR_INVALID_ARG, "unknown flag");
   GemmProblem g{};
   g.mx = fmt == FP4_MXFP4;
   g.A = A;
@@ -237,7 +239,14 @@ fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const floa
   g.out_bf16 = out_dtype == FP4_BF16;
   g.ws = workspace;
   g.ws_bytes = workspace_bytes;
+  g.weights_ready = (flags & FP4_GEMM_WEIGHTS_READY) ? 1 : 0;
   return gemm_common(g, fmt, out_dtype, stream);
+}
+
+fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
+                    const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D, fp4_dtype out_dtype,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace, workspace_bytes, 0u, stream);
 }
 
 fp4_status fp4_gemm_grouped(fp4_fmt fmt, int num_groups, const int32_t* offsets, const uint8_t* A,

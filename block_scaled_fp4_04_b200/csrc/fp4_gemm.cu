@@ -7,21 +7,29 @@
 // epilogue so no extra pass over memory is needed).
 //
 // Structure (one CTA per SM, persistent; 6 warps):
-//   warp 0      TMA producer: per 256-wide K step, one 128x128-byte box of A, one
-//               BNx128-byte box of B (both 128-byte swizzled), and the matching
+//   warp 0      TMA producer: per 256-wide K step, one 128 x 128-byte box of A, one
+//               BN x 128-byte box of B (both 128-byte swizzled), and the matching
 //               512-byte scale-factor atoms by bulk copy, into a STAGES-deep ring.
-//   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale atoms -> TMEM, replicated
-//               to the 4 sub-partitions) and tcgen05.mma.kind::mxf4nvf4 (NVFP4,
+//   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale atoms -> TMEM, replicated to
+//               the 4 sub-partitions) and tcgen05.mma.kind::mxf4nvf4 (NVFP4,
 //               scale_vec::4X, UE4M3) or kind::mxf4 (MXFP4, scale_vec::2X, UE8M0),
 //               M=128, N=BN, K=64 each, accumulating in TMEM; commits free the ring
 //               slot and, at the end of a tile, hand the accumulator to the epilogue.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //               32*(w%4)..+31), multiply by gA*gB, BF16 (RNE) or FP32 store; with
 //               ACC=2 accumulator buffers the epilogue of tile i overlaps tile i+1.
-// Schedules: whole tiles (grouped raster for L2 reuse), stream-K over (tile, K-step)
-// units with FP32 reduction in a workspace (decode shapes, where the small-M problem
-// runs with A and B swapped so the weight rows fill MMA-M), and grouped MoE tiles
-// enumerated on the device from the expert offsets.
+// Schedules: whole tiles (grouped raster for L2 reuse); stream-K over (tile, K-step)
+// units when there are too few tiles to fill the SMs -- each CTA adds its FP32 partial
+// tiles into a workspace with vector reductions and a small finalize kernel applies the
+// global scales, converts, and clears the workspace; grouped MoE tiles enumerated on the
+// device from the expert offsets.
+// Decode-sized M (<= 64) runs with the operands swapped: the weight rows fill MMA-M and
+// the few activation rows are MMA-N (16/32/64), which keeps the tensor-core work held per
+// pipeline stage small and therefore many stages of weights in flight.
+// Scale-factor TMEM addresses are always multiples of 4 columns (one 128-row atom per
+// 4 columns); the hardware faults on other alignments.
+// Launched with programmatic dependent launch: the prologue overlaps the previous
+// kernel; global memory is touched only after griddepcontrol.wait.
 // No TMA multicast is used anywhere.  Every wait is bounded (fp4_ptx.cuh); on a timeout
 // the CTA latches the status word, drains its in-flight copies and MMAs, frees TMEM and
 // returns.
@@ -53,8 +61,8 @@ struct GemmArgs {
   void* out;
   int64_t ldo;
   int out_bf16, transposed, vec_store;
+  int indep;  // 1: kernel A, 2: kernel B may be read before the preceding kernel finishes
   float* ws;
-  int* counters;
   int mode;
   int tiles_m, tiles_n, group_m;
   int64_t total_units;
@@ -168,6 +176,12 @@ struct Sched {
   }
 };
 
+// Small-N tiles (decode) run two CTAs per SM: one thread issues all tcgen05 operations
+// of a CTA, and issue latency (not tensor-pipe capacity) bounds a single issuer, so two
+// issuers per SM double the rate at which weight stages are consumed.
+template <int BN>
+constexpr int ctas_per_sm() { return BN <= 64 ? 2 : 1; }
+
 template <int BN, bool MX, int ACC>
 struct Cfg {
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
@@ -177,8 +191,12 @@ struct Cfg {
   static constexpr int kSFABytes = kAtomsKT * 512;
   static constexpr int kSFBBytes = kNRB * kAtomsKT * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-  static constexpr int kReserve = 1024 /*align*/ + 1024 /*barriers*/ + 2 * (kMaxGroups + 1) * 4;
-  static constexpr int kStagesFit = (227 * 1024 - kReserve) / kStageBytes;
+  static constexpr int kCtasPerSm = ctas_per_sm<BN>();
+  // grouped schedules use 128-wide tiles only, so small-N kernels skip the group tables
+  static constexpr int kGroupBytes = kCtasPerSm == 1 ? 2 * (kMaxGroups + 1) * 4 : 0;
+  static constexpr int kReserve = 1024 /*align*/ + 1024 /*barriers*/ + kGroupBytes;
+  static constexpr int kSmemBudget = kCtasPerSm == 1 ? 227 * 1024 : 113 * 1024;
+  static constexpr int kStagesFit = (kSmemBudget - kReserve) / kStageBytes;
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
   static constexpr int kSmemBytes = kStages * kStageBytes + kReserve;
   static constexpr int kSFACols = kAtomsKT * 4;
@@ -208,18 +226,26 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
-// Stores 16 consecutive columns [col, col+16) of one output row (kernel orientation).
+// Waits until the grids this one depends on (programmatic dependent launch) have
+// finished and their writes are visible; a no-op when launched without the attribute.
+__device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the kernel launched after this one on the stream start its prologue now (it still
+// waits for this grid's completion before it reads what this grid writes).
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void store_out(const GemmArgs& p, int64_t off, float v) {
+  if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[off] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(p.out)[off] = v;
+}
+
+// Stores 16 consecutive kernel columns [col, col+16) of one kernel row.  With swapped
+// operands (transposed) kernel row = output column and kernel column = output row.
 __device__ __forceinline__ void store_row16(const GemmArgs& p, int row, int col, const float (&v)[16]) {
   if (p.transposed) {
-    // kernel row = problem column, kernel column = problem row
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (col + j < p.Nk) {
-        const int64_t off = static_cast<int64_t>(col + j) * p.ldo + row;
-        if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[off] = __float2bfloat16_rn(v[j]);
-        else reinterpret_cast<float*>(p.out)[off] = v[j];
-      }
-    }
+    for (int j = 0; j < 16; ++j)
+      if (col + j < p.Nk) store_out(p, static_cast<int64_t>(col + j) * p.ldo + row, v[j]);
     return;
   }
   const int64_t base = static_cast<int64_t>(row) * p.ldo + col;
@@ -238,16 +264,12 @@ __device__ __forceinline__ void store_row16(const GemmArgs& p, int row, int col,
     return;
   }
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    if (col + j < p.Nk) {
-      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[base + j] = __float2bfloat16_rn(v[j]);
-      else reinterpret_cast<float*>(p.out)[base + j] = v[j];
-    }
-  }
+  for (int j = 0; j < 16; ++j)
+    if (col + j < p.Nk) store_out(p, base + j, v[j]);
 }
 
 template <int BN, bool MX, int ACC>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, ctas_per_sm<BN>())
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmArgs p) {
   using C = Cfg<BN, MX, ACC>;
@@ -262,13 +284,13 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* drain = acc_empty + ACC;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  volatile int* s_last = s_abort + 1;
-  volatile int* s_epi_fail = s_abort + 2;
+  volatile int* s_epi_fail = s_abort + 1;
   int* s_mt = reinterpret_cast<int*>(misc + 1024);
   int* s_off = s_mt + (kMaxGroups + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // prologue (overlaps the tail of the previous kernel under programmatic launch)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -280,11 +302,21 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(drain, 1);
     *s_abort = 0;
-    *s_last = 0;
     *s_epi_fail = 0;
     fence_mbar_init();
   }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  // the finalize kernel (if any) may launch now and wait for this grid to complete
+  allow_dependents();
   if (p.mode == kModeGrouped && warp == 2) {
+    wait_prior_grids();  // the offsets may come from the previous kernel
     // m-tile prefix per group (= scale row-block prefix of the grouped A layout)
     const int E = p.num_groups;
     int carry = 0;
@@ -310,10 +342,6 @@ __global__ void __launch_bounds__(192, 1)
       s_off[E] = p.offsets[E];
     }
   }
-  if (warp == 1) {
-    tmem_alloc(s_tmem, C::kTmemCols);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -323,11 +351,55 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
-      // decode streams the weights once (evict first) and re-reads the tiny activations
+      // swapped decode: the weights (A here) are read once -> evict first; the small
+      // activations (B) are re-read by every CTA -> keep
       const uint64_t pol_a = p.transposed ? l2_policy_evict_first() : l2_policy_normal();
       const uint64_t pol_b = p.transposed ? l2_policy_evict_last() : l2_policy_normal();
+      // Loads of one stage: the A box and A scales ("a" side), the B box and B scales.
+      auto load_side = [&](int st_idx, const Work& w, int kb, bool side_a) {
+        uint8_t* st = smem + st_idx * C::kStageBytes;
+        const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+        const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
+        const int64_t koff = static_cast<int64_t>(kb) * C::kAtomsKT * 512;
+        if (side_a) {
+          tma_load_2d(st, &tmA, &full[st_idx], kb * 128, w.a_row, pol_a);
+          bulk_load(st + C::kABytes + C::kBBytes, p.sfa + w.sfa_rb * p.sfa_rb_bytes + koff, sf_bytes, &full[st_idx],
+                    pol_a);
+        } else {
+          tma_load_2d(st + C::kABytes, &tmB, &full[st_idx], kb * 128, w.b_row, pol_b);
+          const int rb0 = w.n0 / 128;
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; ++rb)
+            if (rb0 + rb < p.sfb_rbs)
+              bulk_load(st + C::kABytes + C::kBBytes + C::kSFABytes + rb * C::kAtomsKT * 512,
+                        p.sfb + w.sfb_off + rb * p.sfb_rb_bytes + koff, sf_bytes, &full[st_idx], pol_b);
+        }
+      };
+      auto stage_bytes = [&](const Work& w, int kb) -> uint32_t {
+        const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+        const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
+        const int rb0 = w.n0 / 128;
+        int nrb = 0;
+#pragma unroll
+        for (int rb = 0; rb < C::kNRB; ++rb) nrb += (rb0 + rb < p.sfb_rbs) ? 1 : 0;
+        return C::kABytes + C::kBBytes + sf_bytes * (1 + nrb);
+      };
+      // With an independent operand, the first ring-full of stages loads only that side,
+      // then waits for the preceding kernel, then issues the other side of those stages.
+      const bool early = p.indep != 0;
+      const bool early_a = p.indep == 1;
+      int npend = 0;
+      bool replayed = !early;
+      auto replay = [&]() {
+        wait_prior_grids();
+        Sched<BN> rs(p, s_mt, s_off);
+        Work rw;
+        int j = 0;
+        while (j < npend && rs.next(rw))
+          for (int kb = rw.kb0; kb < rw.kb1 && j < npend; ++kb, ++j) load_side(j, rw, kb, !early_a);
+        replayed = true;
+      };
+      if (!early) wait_prior_grids();
       Sched<BN> sch(p, s_mt, s_off);
       Work w;
       int stage = 0;
@@ -340,23 +412,14 @@ __global__ void __launch_bounds__(192, 1)
             ok = false;
             break;
           }
-          uint8_t* st = smem + stage * C::kStageBytes;
-          const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
-          const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
-          const int rb0 = w.n0 / 128;
-          int nrb = 0;
-#pragma unroll
-          for (int rb = 0; rb < C::kNRB; ++rb) nrb += (rb0 + rb < p.sfb_rbs) ? 1 : 0;
-          const uint32_t bytes = C::kABytes + C::kBBytes + sf_bytes * (1 + nrb);
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(st, &tmA, &full[stage], kb * 128, w.a_row, pol_a);
-          tma_load_2d(st + C::kABytes, &tmB, &full[stage], kb * 128, w.b_row, pol_b);
-          const int64_t koff = static_cast<int64_t>(kb) * C::kAtomsKT * 512;
-          bulk_load(st + C::kABytes + C::kBBytes, p.sfa + w.sfa_rb * p.sfa_rb_bytes + koff, sf_bytes, &full[stage],
-                    pol_a);
-          for (int rb = 0; rb < nrb; ++rb)
-            bulk_load(st + C::kABytes + C::kBBytes + C::kSFABytes + rb * C::kAtomsKT * 512,
-                      p.sfb + w.sfb_off + rb * p.sfb_rb_bytes + koff, sf_bytes, &full[stage], pol_b);
+          mbar_arrive_expect_tx(&full[stage], stage_bytes(w, kb));
+          if (!replayed) {
+            load_side(stage, w, kb, early_a);
+            if (++npend == S) replay();
+          } else {
+            load_side(stage, w, kb, true);
+            load_side(stage, w, kb, false);
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -365,6 +428,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
+      if (ok && !replayed) replay();
       if (*s_abort) {  // let every issued copy land before the CTA's shared memory goes away
         for (int s = 0; s < S; ++s)
           if (issued & (1u << s)) {
@@ -377,15 +441,14 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       Sched<BN> sch(p, s_mt, s_off);
+      const uint32_t smem_base = smem_u32(smem);
       Work w;
       int stage = 0, iter = 0;
-      uint32_t phase = 0, kb_iter = 0;
+      uint32_t phase = 0, slot = 0;
       bool ok = true;
-      const uint32_t smem_base = smem_u32(smem);
       while (ok && sch.next(w)) {
         const int acc = iter % ACC;
-        const uint32_t acc_par = (iter / ACC) & 1;
-        if (!mbar_wait(&acc_empty[acc], acc_par ^ 1, s_abort)) {
+        if (!mbar_wait(&acc_empty[acc], ((iter / ACC) & 1) ^ 1, s_abort)) {
           latch_timeout(s_abort, p.status);
           break;
         }
@@ -399,7 +462,6 @@ __global__ void __launch_bounds__(192, 1)
           }
           tc_fence_after();
           const uint32_t st = smem_base + stage * C::kStageBytes;
-          const uint32_t slot = kb_iter & 1;
           const uint32_t sfa_t = tmem + sf_col0 + slot * C::kSFSlot;
           const uint32_t sfb_t = sfa_t + C::kSFACols;
           const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
@@ -427,7 +489,7 @@ __global__ void __launch_bounds__(192, 1)
               tc_mma_nvfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
           }
           tc_commit(&empty[stage]);
-          ++kb_iter;
+          slot ^= 1;
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
@@ -445,7 +507,8 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int rl = q * 32 + lane;  // accumulator row (TMEM lane) of this thread
+      const int rl = q * 32 + lane;     // accumulator row (TMEM lane) of this thread
+    wait_prior_grids();               // the global scales come from earlier kernels
     const float ga = p.ga ? *p.ga : 1.0f;
     Sched<BN> sch(p, s_mt, s_off);
     Work w;
@@ -467,62 +530,35 @@ __global__ void __launch_bounds__(192, 1)
       const bool row_ok = rl < w.rows_valid;
       const int row = w.out_row0 + rl;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+      if (q * 32 < w.rows_valid) {  // warp-uniform: warps without a valid row skip TMEM
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(taddr + c, r);
-        tmem_ld_wait();
-        const int col = w.n0 + c;
-        if (!row_ok || col >= p.Nk) continue;
-        if (p.mode == kModeStreamK) {
-          float* dst = p.ws + static_cast<int64_t>(row) * p.Nk + col;
-          if ((p.Nk & 3) == 0 && col + 16 <= p.Nk) {
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c, r);
+          tmem_ld_wait();
+          const int col = w.n0 + c;
+          if (!row_ok || col >= p.Nk) continue;
+          if (p.mode == kModeStreamK) {
+            float* dst = p.ws + static_cast<int64_t>(row) * p.Nk + col;
+            if ((p.Nk & 3) == 0 && col + 16 <= p.Nk) {
 #pragma unroll
-            for (int j = 0; j < 16; j += 4)
-              red_add_v4(dst + j, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                         __uint_as_float(r[j + 3]));
+              for (int j = 0; j < 16; j += 4)
+                red_add_v4(dst + j, __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                           __uint_as_float(r[j + 3]));
+            } else {
+              for (int j = 0; j < 16 && col + j < p.Nk; ++j) atomicAdd(dst + j, __uint_as_float(r[j]));
+            }
           } else {
-            for (int j = 0; j < 16 && col + j < p.Nk; ++j) atomicAdd(dst + j, __uint_as_float(r[j]));
-          }
-        } else {
-          float v[16];
+            float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]) * scale;
-          store_row16(p, row, col, v);
+            for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]) * scale;
+            store_row16(p, row, col, v);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      if (p.mode == kModeStreamK) {
-        // the CTA that completes a tile's K range converts it and clears the workspace
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (warp == 2 && lane == 0) {
-          const int prev = atomicAdd(p.counters + w.tile, w.kb1 - w.kb0);
-          *s_last = (prev + (w.kb1 - w.kb0) == p.num_kb) ? 1 : 0;
-          if (*s_last) p.counters[w.tile] = 0;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (*s_last) {
-          __threadfence();
-          if (row_ok) {
-            for (int c = 0; c < BN; c += 16) {
-              const int col = w.n0 + c;
-              if (col >= p.Nk) break;
-              float* src = p.ws + static_cast<int64_t>(row) * p.Nk + col;
-              float v[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                v[j] = (col + j < p.Nk) ? __ldcg(src + j) * scale : 0.0f;
-                if (col + j < p.Nk) __stcg(src + j, 0.0f);
-              }
-              store_row16(p, row, col, v);
-            }
-          }
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-      }
       ++iter;
     }
   }
@@ -533,6 +569,38 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Stream-K finalize: D = gA * gB * workspace (kernel orientation [Mk, Nk], written back
+// transposed when the operands were swapped), then the workspace is cleared for the next
+// call.  Launched right after the GEMM with programmatic dependent launch.
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(const GemmArgs p) {
+  wait_prior_grids();
+  const float scale = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f);
+  const int nq = (p.Nk + 3) / 4;
+  const int64_t total = static_cast<int64_t>(p.Mk) * nq;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    // consecutive threads take consecutive kernel rows: the transposed stores coalesce
+    const int r = static_cast<int>(idx % p.Mk);
+    const int c = static_cast<int>(idx / p.Mk) * 4;
+    float* src = p.ws + static_cast<int64_t>(r) * p.Nk + c;
+    float v[4];
+    if ((p.Nk & 3) == 0) {
+      const float4 t = __ldcs(reinterpret_cast<const float4*>(src));
+      *reinterpret_cast<float4*>(src) = make_float4(0.f, 0.f, 0.f, 0.f);
+      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+      for (int j = 0; j < 4; ++j) {
+        v[j] = c + j < p.Nk ? src[j] : 0.0f;
+        if (c + j < p.Nk) src[j] = 0.0f;
+      }
+    }
+    for (int j = 0; j < 4 && c + j < p.Nk; ++j) {
+      const int64_t o = p.transposed ? static_cast<int64_t>(c + j) * p.ldo + r : static_cast<int64_t>(r) * p.ldo + c + j;
+      store_out(p, o, v[j] * scale);
+    }
   }
 }
 
@@ -577,9 +645,10 @@ struct Plan {
   size_t ws_bytes;
 };
 
-static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped) {
+static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
   Plan pl{};
   pl.num_kb = static_cast<int>((K + 255) / 256);
+  (void)mx;
   if (grouped) {
     pl.swap = false;
     pl.BN = 128;
@@ -591,7 +660,7 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped) {
     pl.ws_bytes = 0;
     return pl;
   }
-  if (M <= 64) {  // decode: weight rows fill MMA-M, tokens map to MMA-N
+  if (M <= 64) {  // decode: weight rows fill MMA-M, the few activation rows are MMA-N
     pl.swap = true;
     pl.Mk = N;
     pl.Nk = M;
@@ -608,10 +677,11 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped) {
   pl.tiles_n = static_cast<int>((pl.Nk + pl.BN - 1) / pl.BN);
   const int64_t tiles = static_cast<int64_t>(pl.tiles_m) * pl.tiles_n;
   const int sms = num_sms();
-  if (pl.swap || (tiles < sms && pl.num_kb >= 4)) {
+  // too few tiles to fill the SMs: split every tile's K range across CTAs (stream-K)
+  if (tiles < 2 * sms && pl.num_kb >= 4) {
     pl.mode = kModeStreamK;
     pl.units = tiles * pl.num_kb;
-    pl.ws_bytes = static_cast<size_t>(pl.Mk * pl.Nk) * 4 + static_cast<size_t>(tiles) * 4 + 256;
+    pl.ws_bytes = static_cast<size_t>(M * N) * 4;
   } else {
     pl.mode = kModeTile;
     pl.units = tiles;
@@ -620,10 +690,7 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped) {
   return pl;
 }
 
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx) {
-  (void)mx;
-  return make_plan(M, N, K, 0).ws_bytes;
-}
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx) { return make_plan(M, N, K, 0, mx).ws_bytes; }
 
 template <int BN, bool MX, int ACC>
 static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid, cudaStream_t st) {
@@ -631,48 +698,66 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
   auto kern = fp4_gemm_kernel<BN, MX, ACC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 192, C::kSmemBytes, st>>>(ta, tb, a);
-  return cudaGetLastError();
+  // programmatic dependent launch: the prologue (barriers, TMEM, descriptor prefetch)
+  // overlaps the previous kernel on the stream; the kernel waits for it before reading
+  // any global memory
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid * C::kCtasPerSm);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+  if (e != cudaSuccess || a.mode != kModeStreamK) return e;
+  cudaLaunchConfig_t fin = cfg;
+  const int64_t work = static_cast<int64_t>(a.Mk) * ((a.Nk + 3) / 4);
+  fin.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * num_sms()))));
+  fin.blockDim = dim3(256);
+  fin.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&fin, splitk_finalize_kernel, a);
 }
 
 template <bool MX>
-static cudaError_t dispatch(int BN, int ACC, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                            int grid, cudaStream_t st) {
-  switch (BN) {
+static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid,
+                            cudaStream_t st) {
+  switch (pl.BN) {
     case 16: return run<16, MX, 2>(ta, tb, a, grid, st);
     case 32: return run<32, MX, 2>(ta, tb, a, grid, st);
     case 64: return run<64, MX, 2>(ta, tb, a, grid, st);
     case 128: return run<128, MX, 2>(ta, tb, a, grid, st);
-    default: return ACC == 1 ? run<256, MX, 1>(ta, tb, a, grid, st) : cudaErrorInvalidValue;
+    default: return run<256, MX, 1>(ta, tb, a, grid, st);
   }
 }
 
 int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err) {
   const int grouped = g.num_groups > 0;
-  const Plan pl = make_plan(g.M, g.N, g.K, grouped);
+  const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx);
   if (g.ws_bytes < pl.ws_bytes || (pl.ws_bytes && !g.ws)) {
     *why = "workspace too small (see fp4_gemm_workspace_size)";
     return 1;
   }
   const int64_t sf_cols = g.K / (g.mx ? 32 : 16);
   const int64_t atoms_k = (sf_cols + 3) / 4;
-  GemmArgs a{};
   const uint8_t *kA = g.A, *kB = g.B, *kSA = g.sA, *kSB = g.sB;
   const float *kgA = g.gA, *kgB = g.gB;
-  int64_t rowsA = g.M, rowsB = g.N;
+  int64_t rowsA = g.M, rowsB = grouped ? static_cast<int64_t>(g.num_groups) * g.N : g.N;
   if (pl.swap) {
     std::swap(kA, kB);
     std::swap(kSA, kSB);
     std::swap(kgA, kgB);
     std::swap(rowsA, rowsB);
   }
-  if (grouped) rowsB = static_cast<int64_t>(g.num_groups) * g.N;
   CUtensorMap ta, tb;
   if (!make_map(&ta, kA, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsA), 128) ||
       !make_map(&tb, kB, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsB), static_cast<uint32_t>(pl.BN))) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
     return 1;
   }
+  GemmArgs a{};
   a.sfa = kSA;
   a.sfb = kSB;
   a.sfa_rb_bytes = atoms_k * 512;
@@ -687,7 +772,9 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   a.out = g.D;
   a.out_bf16 = g.out_bf16;
   a.transposed = pl.swap ? 1 : 0;
-  a.ldo = pl.swap ? g.N : g.N;
+  // the weights (problem B) are kernel A when the operands are swapped
+  a.indep = g.weights_ready ? (pl.swap ? 1 : 2) : 0;
+  a.ldo = g.N;
   const int esz = g.out_bf16 ? 2 : 4;
   a.vec_store = ((g.N * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(g.D) & 15) == 0) ? 1 : 0;
   a.mode = pl.mode;
@@ -698,7 +785,6 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   a.status = status;
   if (pl.mode == kModeStreamK) {
     a.ws = static_cast<float*>(g.ws);
-    a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(g.ws) + static_cast<size_t>(pl.Mk * pl.Nk) * 4);
   }
   if (grouped) {
     a.num_groups = g.num_groups;
@@ -709,12 +795,13 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   } else {
     a.sfb_rbs = static_cast<int>((rowsB + 127) / 128);
   }
+  // CTAs per SM are applied by run(); a tile schedule never launches more CTAs than units
   int grid;
+  const int per_sm = pl.BN <= 64 ? 2 : 1;
   if (pl.mode == kModeGrouped) grid = num_sms();
-  else grid = static_cast<int>(std::min<int64_t>(pl.units, num_sms()));
+  else grid = static_cast<int>(std::min<int64_t>((pl.units + per_sm - 1) / per_sm, num_sms()));
   grid = std::max(grid, 1);
-  const cudaError_t e = g.mx ? dispatch<true>(pl.BN, pl.ACC, ta, tb, a, grid, st)
-                             : dispatch<false>(pl.BN, pl.ACC, ta, tb, a, grid, st);
+  const cudaError_t e = g.mx ? dispatch<true>(pl, ta, tb, a, grid, st) : dispatch<false>(pl, ta, tb, a, grid, st);
   if (e != cudaSuccess) {
     *err = e;
     return 2;

@@ -44,6 +44,7 @@ struct GemmProblem {
   int out_bf16;
   void* ws;
   size_t ws_bytes;
+  int weights_ready;         // B was not written by the kernel just before this call
   // grouped
   int num_groups;            // 0: plain GEMM
   const int32_t* offsets;

@@ -59,6 +59,12 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 
 __device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
+// Programmatic dependent launch: let the next kernel on the stream start its prologue
+// early / wait until the previous kernel's writes are visible (no-ops without the
+// launch attribute).
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ amax
 // Grid-stride max of |x| (as bit patterns: for non-negative floats the integer order is
 // the numeric order, and inf / NaN patterns exceed every finite one).  Each block writes
@@ -67,6 +73,7 @@ __device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v
 template <typename T>
 __global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, int64_t n, uint32_t* ws,
                                                     float* amax_out, float* g_out, unsigned* status) {
+  allow_dependents();
   constexpr int EPC = Elem<T>::kPerChunk;
   const int64_t nchunks = n / EPC;
   const uint4* xc = reinterpret_cast<const uint4*>(x);
@@ -200,6 +207,8 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   __shared__ int s_rb[kMaxGroups + 1];
   __shared__ int s_off[kMaxGroups + 1];
 
+  allow_dependents();
+  wait_prior_grids();  // g (and x, offsets) may come from the kernels just before
   const int E = p.offsets ? p.num_groups : 1;
   if (p.offsets) {
     group_prefix(p.offsets, E, s_rb, s_off);
@@ -502,8 +511,16 @@ cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float*
 template <typename T, int BLOCK, bool MX>
 static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
   const int blocks = blocks_for(a.rb_upper * a.ct_count, 8);
-  quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware><<<blocks, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware>, a);
 }
 
 cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,

@@ -145,6 +145,19 @@ fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, co
                     int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,
                     void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* fp4_gemm with options.  flags is a bitwise OR of:
+ *   FP4_GEMM_WEIGHTS_READY  B, sB and gB were written before the kernel that runs just
+ *       before this call on `stream` (for example pre-quantized weights).  The GEMM may
+ *       then start streaming B while that kernel (typically the activation quantize)
+ *       is still running; A and its scales are read only after it has finished.  Setting
+ *       the flag when B is produced by the immediately preceding kernel is a data race.
+ * Unknown bits return FP4_ERR_INVALID_ARG. */
+#define FP4_GEMM_WEIGHTS_READY 1u
+fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,
+                       const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
+                       int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,
+                       void* workspace_dev, size_t workspace_bytes, unsigned flags, void* stream);
+
 /* Grouped (MoE) GEMM ("FP4" glossary entry, inference passage: MoE weights kept in
  * MXFP4): for each group e, rows [offsets[e], offsets[e+1]) of A times expert e's
  * weights B_dev + e*N*K/2 give the same rows of D:

@@ -96,6 +96,12 @@ def test_gemm_rejects_bad_arguments():
                               None, 0, None) == fp4.ERR_INVALID_ARG   # N % 128
 
 
+def test_gemm_ex_rejects_unknown_flags():
+    L = fp4.lib()
+    assert L.fp4_gemm_ex(fp4.NVFP4, 16, 16, 16, 16, 16, 16, 128, 128, 256, 16, fp4.BF16, None, 0, 6, None) \
+        == fp4.ERR_INVALID_ARG
+
+
 def test_last_error_message():
     _rc_quantize(cols=48)
     assert b"multiple of 32" in fp4.lib().fp4_last_error()

@@ -190,3 +190,25 @@ def test_training_weight_reuse_forward_and_backward():
     assert np.array_equal(w_hat.T, wT_hat)
     check_gemm(d, dequant_oracle(oracle_quantize(x, fp4.NVFP4, 16), fp4.NVFP4), w_hat, label="fwd")
     check_gemm(dx, dequant_oracle(oracle_quantize(dy, fp4.NVFP4, 16), fp4.NVFP4), wT_hat, label="bwd")
+
+
+def test_gemm_ex_weights_ready_decode():
+    """Activations quantized by the kernel just before the GEMM; the weights were quantized
+    earlier, so the GEMM may stream them before the activation quantize has finished."""
+    m, n, k = 16, 4096, 8192
+    xa = random_input(m, k, 77, torch.bfloat16)
+    xb = random_input(n, k, 78, torch.float32, std=0.02, outliers=False)
+    qb = gpu_quantize(xb.cuda(), fp4.NVFP4, 16)
+    ws = fp4.Workspace()
+    wsn = fp4.fp4_gemm_workspace_size(m, n, k, fp4.NVFP4)
+    buf = ws.get(wsn)
+    ob = oracle_quantize(xb, fp4.NVFP4, 16)
+    for rep in range(3):
+        qa = fp4.quantize(xa.cuda(), fp4.NVFP4, 16)   # no synchronization in between
+        d = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+        fp4.fp4_gemm_ex(fp4.NVFP4, qa.codes, qa.scales, qa.g, qb.codes, qb.scales, qb.g, m, n, k, d, fp4.BF16,
+                        buf, buf.numel(), fp4.GEMM_WEIGHTS_READY)
+        torch.cuda.synchronize()
+        assert fp4.fp4_get_status() == fp4.OK
+        oa = oracle_quantize(xa, fp4.NVFP4, 16)
+        check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label=f"rep {rep}")
