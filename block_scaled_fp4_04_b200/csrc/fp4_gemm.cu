@@ -576,6 +576,7 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
 // transposed when the operands were swapped), then the workspace is cleared for the next
 // call.  Launched right after the GEMM with programmatic dependent launch.
 __global__ void __launch_bounds__(256) splitk_finalize_kernel(const GemmArgs p) {
+  allow_dependents();  // the next kernel may launch; it waits for this grid before using D
   wait_prior_grids();
   const float scale = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f);
   const int nq = (p.Nk + 3) / 4;
@@ -624,7 +625,7 @@ static EncodeTiledFn encode_fn() {
 
 // [rows, inner_bytes] uint8 matrix, boxes of box_rows x 128 bytes, 128-byte swizzle,
 // out-of-bounds elements read as zero.
-static bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+static bool encode_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner_bytes, rows};
@@ -634,6 +635,43 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uin
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Small host cache of encoded tensor maps keyed by (address, shape, box): decode-style
+// callers pass the same buffers every step, and encoding costs host time on every call.
+// A map only describes addresses, so a stale entry is just another valid encoding.
+struct MapCacheEntry {
+  const void* base;
+  uint64_t inner, rows;
+  uint32_t box;
+  CUtensorMap map;
+};
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+  constexpr int kEntries = 32;
+  static MapCacheEntry cache[kEntries];
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const MapCacheEntry& e = cache[i];
+      if (e.base == base && e.inner == inner_bytes && e.rows == rows && e.box == box_rows) {
+        *m = e.map;
+        return true;
+      }
+    }
+  }
+  if (!encode_map(m, base, inner_bytes, rows, box_rows)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  MapCacheEntry& e = cache[next];
+  e.base = base;
+  e.inner = inner_bytes;
+  e.rows = rows;
+  e.box = box_rows;
+  e.map = *m;
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  return true;
 }
 
 struct Plan {
@@ -696,8 +734,16 @@ template <int BN, bool MX, int ACC>
 static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid, cudaStream_t st) {
   using C = Cfg<BN, MX, ACC>;
   auto kern = fp4_gemm_kernel<BN, MX, ACC>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
+  // the shared-memory opt-in is per device; set it once per (kernel, device)
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t e = cudaSuccess;
+  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_done[dev] = true;
+  }
   // programmatic dependent launch: the prologue (barriers, TMEM, descriptor prefetch)
   // overlaps the previous kernel on the stream; the kernel waits for it before reading
   // any global memory

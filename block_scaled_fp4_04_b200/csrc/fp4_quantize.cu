@@ -74,6 +74,7 @@ template <typename T>
 __global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, int64_t n, uint32_t* ws,
                                                     float* amax_out, float* g_out, unsigned* status) {
   allow_dependents();
+  wait_prior_grids();  // x may be the output of the kernel just before
   constexpr int EPC = Elem<T>::kPerChunk;
   const int64_t nchunks = n / EPC;
   const uint4* xc = reinterpret_cast<const uint4*>(x);
@@ -500,12 +501,19 @@ cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float*
   const int64_t chunks = (n + epc - 1) / epc;
   int blocks = static_cast<int>(std::min<int64_t>((chunks + 2047) / 2048, static_cast<int64_t>(num_sms()) * 4));
   blocks = std::max(1, std::min(blocks, kAmaxMaxBlocks));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(512);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (bf16)
-    amax_kernel<__nv_bfloat16><<<blocks, 512, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n, ws, amax_out,
-                                                        g_out, status);
-  else
-    amax_kernel<float><<<blocks, 512, 0, st>>>(static_cast<const float*>(x), n, ws, amax_out, g_out, status);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, amax_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x), n, ws, amax_out,
+                              g_out, status);
+  return cudaLaunchKernelEx(&cfg, amax_kernel<float>, static_cast<const float*>(x), n, ws, amax_out, g_out, status);
 }
 
 template <typename T, int BLOCK, bool MX>
