@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
                 "fp4_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
                 "fp4_gemm": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_gemm_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, ctypes.c_uint, P]),
+                "fp4_gemm_noalloc": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
                 "fp4_gemm_grouped": (I32, [I32, I32, P, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_get_status": (I32, [P]),
                 "fp4_debug_encode": (I32, [P, I64, I32, P, P]),
@@ -160,6 +161,13 @@ def fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace=None
                 stream=None):
     _check(lib().fp4_gemm_ex(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype,
                              _p(workspace), workspace_bytes, flags, _s(stream)))
+
+
+def fp4_gemm_noalloc(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, stream=None):
+    """fp4_gemm without a caller workspace: the split-K scratch is a fixed 4 MiB array
+    inside the library, shared by all calls on a device (calls that overlap race)."""
+    _check(lib().fp4_gemm_noalloc(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype,
+                                  _s(stream)))
 
 
 def fp4_gemm_grouped(fmt, num_groups, offsets, A, sA, gA, B, sB, gB, total_rows, N, K, D, out_dtype,

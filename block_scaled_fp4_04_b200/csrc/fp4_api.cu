@@ -249,6 +249,66 @@ fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const floa
   return fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace, workspace_bytes, 0u, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Allocation-free GEMM.  Callers that cannot allocate device memory -- code running
+// while a CUDA graph is being captured, or a host (plugin runtime, embedded engine)
+// that owns every device byte and hands this library no allocator -- still need the
+// split-K scratch that decode-sized GEMMs use.  This variant takes it from a fixed
+// array compiled into the library instead of from the caller.
+namespace fp4 {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB on every device that loads the library
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on the current device.  The array's host-side name is
+// only a stand-in; the device address comes from cudaGetSymbolAddress, done once per
+// device with that device current (the first call on a device does it, so make that
+// first call before any stream capture).
+static fp4_status noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP4_ERR_UNSUPPORTED, "device index out of range");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FP4_OK;
+}
+}  // namespace fp4
+
+extern "C" {
+
+fp4_status fp4_gemm_noalloc(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
+                            const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D,
+                            fp4_dtype out_dtype, void* stream) {
+  if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "fmt");
+  const size_t need = (M > 0 && N > 0 && K > 0) ? gemm_workspace_bytes(M, N, K, fmt == FP4_MXFP4) : 0;
+  if (need > kNoAllocScratchBytes) {
+    snprintf(g_err, sizeof(g_err),
+             "fp4_gemm_noalloc: this shape needs %zu bytes of scratch but the built-in array holds %zu "
+             "(4 MiB); use fp4_gemm with a caller workspace",
+             need, kNoAllocScratchBytes);
+    return FP4_ERR_INVALID_ARG;
+  }
+  void* ws = nullptr;
+  if (need) {
+    fp4_status s = noalloc_scratch(&ws);
+    if (s != FP4_OK) return s;
+    // every call shares the array: clear the part this call accumulates into
+    cudaError_t e = cudaMemsetAsync(ws, 0, need, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the no-alloc scratch");
+  }
+  return fp4_gemm(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, ws, need, stream);
+}
+
 fp4_status fp4_gemm_grouped(fp4_fmt fmt, int num_groups, const int32_t* offsets, const uint8_t* A,
                             const uint8_t* sA, const float* gA, const uint8_t* B, const uint8_t* sB,
                             const float* gB, int64_t total_rows, int64_t N, int64_t K, void* D,
