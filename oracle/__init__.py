@@ -43,16 +43,53 @@ F32 = 0
 BF16 = 1
 ERR_NONFINITE = 5
 
+# IEEE single-precision arithmetic as written: no FMA contraction, no fast-math.
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-Wall", "-fopenmp", "-shared", "-fPIC"]
+
 
 def build(force: bool = False) -> str:
     """Compile fp4_oracle.c into oracle/liboracle.so with gcc (no FMA contraction)."""
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.check_call(
-            ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-Wall", "-fopenmp",
-             "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
+
+
+def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declares the C functions' signatures on a loaded copy of the oracle library."""
+    P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sig = {
+        "orc_e2m1_decode": (ctypes.c_double, [ctypes.c_uint8]),
+        "orc_e2m1_encode": (ctypes.c_uint8, [ctypes.c_float]),
+        "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
+        "orc_e4m3_encode": (ctypes.c_uint8, [ctypes.c_float]),
+        "orc_e8m0_decode": (ctypes.c_double, [ctypes.c_uint8]),
+        "orc_e8m0_encode": (ctypes.c_uint8, [ctypes.c_float]),
+        "orc_e2m1_encode_array": (None, [P, I64, P]),
+        "orc_e4m3_encode_array": (None, [P, I64, P]),
+        "orc_e8m0_encode_array": (None, [P, I64, P]),
+        "orc_amax": (I32, [P, I64, I32, P]),
+        "orc_global_scale": (ctypes.c_float, [ctypes.c_float]),
+        "orc_quantize_nvfp4_1d": (I32, [P, I64, I64, I32, P, P, P, P]),
+        "orc_quantize_mxfp4_1d": (I32, [P, I64, I64, I32, P, P]),
+        "orc_quantize_nvfp4_2d": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
+        "orc_scales_bytes": (I64, [I64, I64]),
+        "orc_swizzle_offset": (I64, [I64, I64, I64]),
+        "orc_swizzle_scales": (None, [P, I64, I64, P]),
+        "orc_unswizzle_scales": (None, [P, I64, I64, P]),
+        "orc_scales_bytes_grouped": (I64, [P, I32, I64]),
+        "orc_swizzle_scales_grouped": (None, [P, P, I32, I64, P]),
+        "orc_dequantize": (None, [P, P, ctypes.c_float, I64, I64, I32, P]),
+        "orc_fake_quant_fp32_scale": (None, [P, I64, I64, P]),
+        "orc_e2m1_count_mismatch": (I64, [ctypes.c_uint64, I64, P]),
+        "orc_num_threads": (I32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
 
 
 def _L():
@@ -60,39 +97,7 @@ def _L():
     with _lock:
         if _lib is None:
             build()
-            lib = ctypes.CDLL(_LIB_PATH)
-            P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-            sig = {
-                "orc_e2m1_decode": (ctypes.c_double, [ctypes.c_uint8]),
-                "orc_e2m1_encode": (ctypes.c_uint8, [ctypes.c_float]),
-                "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
-                "orc_e4m3_encode": (ctypes.c_uint8, [ctypes.c_float]),
-                "orc_e8m0_decode": (ctypes.c_double, [ctypes.c_uint8]),
-                "orc_e8m0_encode": (ctypes.c_uint8, [ctypes.c_float]),
-                "orc_e2m1_encode_array": (None, [P, I64, P]),
-                "orc_e4m3_encode_array": (None, [P, I64, P]),
-                "orc_e8m0_encode_array": (None, [P, I64, P]),
-                "orc_amax": (I32, [P, I64, I32, P]),
-                "orc_global_scale": (ctypes.c_float, [ctypes.c_float]),
-                "orc_quantize_nvfp4_1d": (I32, [P, I64, I64, I32, P, P, P, P]),
-                "orc_quantize_mxfp4_1d": (I32, [P, I64, I64, I32, P, P]),
-                "orc_quantize_nvfp4_2d": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
-                "orc_scales_bytes": (I64, [I64, I64]),
-                "orc_swizzle_offset": (I64, [I64, I64, I64]),
-                "orc_swizzle_scales": (None, [P, I64, I64, P]),
-                "orc_unswizzle_scales": (None, [P, I64, I64, P]),
-                "orc_scales_bytes_grouped": (I64, [P, I32, I64]),
-                "orc_swizzle_scales_grouped": (None, [P, P, I32, I64, P]),
-                "orc_dequantize": (None, [P, P, ctypes.c_float, I64, I64, I32, P]),
-                "orc_fake_quant_fp32_scale": (None, [P, I64, I64, P]),
-                "orc_e2m1_count_mismatch": (I64, [ctypes.c_uint64, I64, P]),
-                "orc_num_threads": (I32, []),
-            }
-            for name, (res, args) in sig.items():
-                fn = getattr(lib, name)
-                fn.restype = res
-                fn.argtypes = args
-            _lib = lib
+            _lib = configure(ctypes.CDLL(_LIB_PATH))
     return _lib
 
 

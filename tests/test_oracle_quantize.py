@@ -110,6 +110,22 @@ def test_error_bound_unsaturated():
     assert np.all(np.abs(x - xh)[ok] <= (0.5 * gap * s * (1 + 1e-6))[ok])
 
 
+def test_no_element_beyond_the_block_range():
+    """The block scale covers the block's largest magnitude: with a normal E4M3 scale
+    below the 448 clamp, sb = E4M3(amax_b / (6 g)) is within half an E4M3 ulp (2^-4
+    relative) of its argument, so every |x| / (dec(sb) g) <= 6 (1 + 2^-4).  For MXFP4
+    the power of two rounds amax_b / 6 by at most a factor 1.5: |x| / dec(sb) < 9."""
+    x = _rand(64, 512, 12)
+    q = oracle.quantize(x, oracle.NVFP4, 16)
+    s = np.repeat(np.array([[oracle.e4m3_decode(c) for c in row] for row in q["scales"]]), 16, 1)
+    normal = np.repeat((q["scales"] >= 8) & (q["scales"] < 0x7E), 16, 1)
+    r = np.abs(x) / (s * float(q["g"]))
+    assert normal.mean() > 0.9 and np.all(r[normal] <= 6 * (1 + 2.0 ** -4))
+    m = oracle.quantize(x, oracle.MXFP4, 32)
+    sm = np.repeat(np.array([[oracle.e8m0_decode(c) for c in row] for row in m["scales"]]), 32, 1)
+    assert np.all(np.abs(x) / sm < 9.0)
+
+
 def test_global_scale():
     assert oracle.global_scale(2688.0) == 1.0
     assert oracle.global_scale(0.0) == 1.0
