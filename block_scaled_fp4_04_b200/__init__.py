@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
                 "fp4_gemm": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_gemm_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_noalloc": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
+                "fp4_gemm_bf16a_workspace_size": (SZ, [I64, I64, I64]),
+                "fp4_gemm_bf16a": (I32, [P, P, P, P, I64, I64, I64, P, I32, P, P, P, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_grouped": (I32, [I32, I32, P, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_get_status": (I32, [P]),
                 "fp4_debug_encode": (I32, [P, I64, I32, P, P]),
@@ -161,6 +163,16 @@ def fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace=None
                 stream=None):
     _check(lib().fp4_gemm_ex(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype,
                              _p(workspace), workspace_bytes, flags, _s(stream)))
+
+
+def fp4_gemm_bf16a_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib().fp4_gemm_bf16a_workspace_size(M, N, K))
+
+
+def fp4_gemm_bf16a(X, B, sB, gB, M, N, K, D, out_dtype, Xcodes, Xscales, gX, workspace, workspace_bytes, flags=0,
+                   stream=None):
+    _check(lib().fp4_gemm_bf16a(_p(X), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype, _p(Xcodes), _p(Xscales),
+                                _p(gX), _p(workspace), workspace_bytes, flags, _s(stream)))
 
 
 def fp4_gemm_noalloc(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, stream=None):

@@ -138,8 +138,14 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   if (s != FP4_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bf16 = in_dtype == FP4_BF16;
-  const float* g = nullptr;
+  const int mx = fmt == FP4_MXFP4;
   cudaError_t e = cudaSuccess;
+  if (!two_d && !num_groups && quantize_small_fits(rows, cols, bf16, mx)) {
+    // one launch: amax, global scale and encode by one thread-block cluster
+    e = launch_quantize_small(x, rows, cols, bf16, mx, codes, scales, mx ? nullptr : gin, gout, status, st);
+    return e == cudaSuccess ? FP4_OK : cuda_fail(e, "quantize launch");
+  }
+  const float* g = nullptr;
   if (fmt == FP4_NVFP4) {
     if (need_amax) {
       e = launch_amax(x, rows * cols, bf16, static_cast<uint32_t*>(ws), nullptr, gout, status, st);
@@ -159,7 +165,7 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   if (two_d)
     e = launch_quantize_2d(x, rows, cols, bf16, codes, scales, codesT, scalesT, g, status, st);
   else
-    e = launch_quantize_1d(x, rows, cols, bf16, fmt == FP4_MXFP4, codes, scales, g, offsets, num_groups, status, st);
+    e = launch_quantize_1d(x, rows, cols, bf16, mx, codes, scales, g, offsets, num_groups, status, st);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "quantize launch");
 }
 
@@ -247,6 +253,62 @@ fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const floa
                     const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D, fp4_dtype out_dtype,
                     void* workspace, size_t workspace_bytes, void* stream) {
   return fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace, workspace_bytes, 0u, stream);
+}
+
+size_t fp4_gemm_bf16a_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return gemm_bf16a_workspace_bytes(M, N, K);
+}
+
+fp4_status fp4_gemm_bf16a(const void* X, const uint8_t* B, const uint8_t* sB, const float* gB, int64_t M, int64_t N,
+                          int64_t K, void* D, fp4_dtype out_dtype, uint8_t* Xcodes, uint8_t* Xscales, float* gX,
+                          void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+  if (!X || !B || !sB || !D || !Xcodes || !Xscales || !gX || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "shape (K % 32 == 0)");
+  if (out_dtype != FP4_F32 && out_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "out_dtype");
+  if (flags & ~static_cast<unsigned>(FP4_GEMM_WEIGHTS_READY)) return fail(FP4_ERR_INVALID_ARG, "unknown flag");
+  if (!aligned16(X) || !aligned16(B) || !aligned16(sB) || !aligned16(D) || !aligned16(Xcodes) || !aligned16(Xscales) ||
+      !aligned16(workspace))
+    return fail(FP4_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  if (workspace_bytes < gemm_bf16a_workspace_bytes(M, N, K))
+    return fail(FP4_ERR_INVALID_ARG, "workspace too small (see fp4_gemm_bf16a_workspace_size)");
+  const size_t qws = (kQuantWorkspaceBytes + 255) / 256 * 256;
+  if (decode_eligible(M, N, K)) {
+    // one launch: every CTA derives the activations' global scale and quantizes its K
+    // segment of them itself while its weight stages stream in
+    unsigned* status;
+    const fp4_status ds = device_state(&status);
+    if (ds != FP4_OK) return ds;
+    DecodeProblem q{};
+    q.W = B;
+    q.sW = sB;
+    q.gW = gB;
+    q.X = X;
+    q.Xq_out = Xcodes;
+    q.Xs_out = Xscales;
+    q.gX_out = gX;
+    q.M = M;
+    q.N = N;
+    q.K = K;
+    q.D = D;
+    q.out_bf16 = out_dtype == FP4_BF16;
+    q.ws = static_cast<uint8_t*>(workspace) + qws;
+    q.ws_bytes = workspace_bytes - qws;
+    q.weights_ready = (flags & FP4_GEMM_WEIGHTS_READY) ? 1 : 0;
+    const char* why = nullptr;
+    cudaError_t err = cudaSuccess;
+    const int rc = launch_decode(q, status, static_cast<cudaStream_t>(stream), &why, &err);
+    if (rc == 1) return fail(FP4_ERR_INVALID_ARG, why);
+    if (rc == 2) return cuda_fail(err, "decode GEMM launch");
+    return FP4_OK;
+  }
+  // larger M: the activations' amax and codes, then the GEMM, chained by programmatic
+  // dependent launch (FP4_GEMM_WEIGHTS_READY lets the GEMM stream the weights early)
+  const fp4_status s = fp4_quantize(X, M, K, FP4_BF16, FP4_NVFP4, 16, Xcodes, Xscales, gX, nullptr, nullptr, nullptr, workspace,
+                   kQuantWorkspaceBytes, stream);
+  if (s != FP4_OK) return s;
+  return fp4_gemm_ex(FP4_NVFP4, Xcodes, Xscales, gX, B, sB, gB, M, N, K, D, out_dtype,
+                     static_cast<uint8_t*>(workspace) + qws, workspace_bytes - qws, flags, stream);
 }
 
 }  // extern "C"

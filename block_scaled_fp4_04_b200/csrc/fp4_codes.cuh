@@ -122,4 +122,14 @@ __device__ __forceinline__ float e2m1_value(uint32_t code) {
   return (code & 8u) ? -mag : mag;
 }
 
+// NVFP4 block scale for a block with largest magnitude amax_b under global scale g:
+// sb = E4M3((amax_b / 6) / g) (two IEEE divisions, in that order); returns the element
+// multiplier 1 / (dec(sb) * g) (IEEE reciprocal), or 0 when that denominator is 0.
+__device__ __forceinline__ float nvfp4_block_scale(float amax_b, float g, uint32_t& sb) {
+  const float t = __fdiv_rn(amax_b, 6.0f);
+  sb = e4m3_code(__fdiv_rn(t, g));
+  const float denom = __fmul_rn(e4m3_value(sb), g);
+  return denom == 0.0f ? 0.0f : __frcp_rn(denom);
+}
+
 }  // namespace fp4

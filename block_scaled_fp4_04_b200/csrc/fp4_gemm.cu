@@ -40,6 +40,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "fp4_codes.cuh"
 #include "fp4_internal.h"
 #include "fp4_ptx.cuh"
 
@@ -62,7 +63,8 @@ struct GemmArgs {
   int64_t ldo;
   int out_bf16, transposed, vec_store;
   int indep;  // 1: kernel A, 2: kernel B may be read before the preceding kernel finishes
-  float* ws;
+  float* ws;        // stream-K: FP32 partial sums [Mk, Nk], zero between calls
+  int* tile_cnt;    // stream-K: K steps summed so far per tile, zero between calls
   int mode;
   int tiles_m, tiles_n, group_m;
   int64_t total_units;
@@ -92,18 +94,21 @@ struct Sched {
   int64_t u, u_end;  // stream-K: current / end unit; tile modes: current unit
   int64_t total;
 
-  __device__ Sched(const GemmArgs& args, const int* mt, const int* off) : p(args), s_mt(mt), s_off(off) {
+  int vgrid;         // pipelines in the grid; this one is number vb
+  // vb / vg: this pipeline's index among all pipelines of the grid, and their count
+  __device__ Sched(const GemmArgs& args, const int* mt, const int* off, int vb, int vg)
+      : p(args), s_mt(mt), s_off(off), vgrid(vg) {
     if (p.mode == kModeStreamK) {
-      const int64_t T = p.total_units, G = gridDim.x;
-      u = T * blockIdx.x / G;
-      u_end = T * (blockIdx.x + 1) / G;
+      const int64_t T = p.total_units;
+      u = T * vb / vg;
+      u_end = T * (vb + 1) / vg;
       total = T;
     } else if (p.mode == kModeGrouped) {
       total = static_cast<int64_t>(s_mt[p.num_groups]) * p.tiles_n;
-      u = blockIdx.x;
+      u = vb;
     } else {
       total = p.total_units;
-      u = blockIdx.x;
+      u = vb;
     }
   }
 
@@ -124,7 +129,7 @@ struct Sched {
     }
     if (u >= total) return false;
     const int64_t cur = u;
-    u += gridDim.x;
+    u += vgrid;
     if (p.mode == kModeGrouped) {
       const int E = p.num_groups;
       int lo = 0, hi = E - 1;  // last group e with s_mt[e] * tiles_n <= cur
@@ -176,36 +181,51 @@ struct Sched {
   }
 };
 
-// Small-N tiles (decode) run two CTAs per SM: one thread issues all tcgen05 operations
-// of a CTA, and issue latency (not tensor-pipe capacity) bounds a single issuer, so two
-// issuers per SM double the rate at which weight stages are consumed.
+// Small-N tiles (decode) run two independent pipelines per CTA ("sub-CTAs" of 192
+// threads, each with its own producer, MMA issuer, epilogue warps, shared-memory ring
+// and TMEM columns).  One thread issues all tcgen05 operations of a pipeline, and at
+// N = 16..64 the issue latency of that thread -- not the tensor pipe -- bounds how fast
+// weight stages are consumed, so two issuers per SM double the rate.  (Two CTAs per SM
+// would do the same, but a kernel that allocates TMEM is scheduled one CTA per SM.)
+#ifndef FP4_SMALL_N_PIPES
+#define FP4_SMALL_N_PIPES 2
+#endif
 template <int BN>
-constexpr int ctas_per_sm() { return BN <= 64 ? 2 : 1; }
+constexpr int pipes_per_cta() { return BN <= 32 ? FP4_SMALL_N_PIPES : BN <= 64 ? 2 : 1; }
 
 template <int BN, bool MX, int ACC>
 struct Cfg {
+  static constexpr int kP = pipes_per_cta<BN>();
+  static constexpr int kThreads = 192 * kP;
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSFABytes = kAtomsKT * 512;
   static constexpr int kSFBBytes = kNRB * kAtomsKT * 512;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-  static constexpr int kCtasPerSm = ctas_per_sm<BN>();
-  // grouped schedules use 128-wide tiles only, so small-N kernels skip the group tables
-  static constexpr int kGroupBytes = kCtasPerSm == 1 ? 2 * (kMaxGroups + 1) * 4 : 0;
-  static constexpr int kReserve = 1024 /*align*/ + 1024 /*barriers*/ + kGroupBytes;
-  static constexpr int kSmemBudget = kCtasPerSm == 1 ? 227 * 1024 : 113 * 1024;
-  static constexpr int kStagesFit = (kSmemBudget - kReserve) / kStageBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // a multiple of 1024
+  // grouped schedules use 128-wide tiles only, so multi-pipeline kernels skip the group tables
+  static constexpr int kGroupBytes = kP == 1 ? 2 * (kMaxGroups + 1) * 4 : 0;
+  static constexpr int kMiscBytes = 1024 /*barriers, flags*/ + kGroupBytes;
+  // the opt-in limit per block, less the alignment slack and the static shared memory
+  static constexpr int kSmemLimit = 227 * 1024 - 1024 - 256;
+  static constexpr int kStagesFit = (kSmemLimit / kP - kMiscBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kReserve;
+  // one pipeline's share; the next pipeline's stages start 1024-byte aligned
+  static constexpr int kSubBytes = (kStages * kStageBytes + kMiscBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmemBytes = kP == 1 ? kStages * kStageBytes + kMiscBytes + 1024 : kP * kSubBytes + 1024;
+  static_assert(kSmemBytes + 256 <= 227 * 1024, "shared memory opt-in limit");
   static constexpr int kSFACols = kAtomsKT * 4;
   static constexpr int kSFBCols = kNRB * kAtomsKT * 4;
   static constexpr int kSFSlot = kSFACols + kSFBCols;
   static constexpr int kColsUsed = ACC * BN + 2 * kSFSlot;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
-                                   : kColsUsed <= 256 ? 256 : 512;
-  static_assert(kColsUsed <= 512, "TMEM budget");
+                                   : kColsUsed <= 256 ? 256 : 512;  // per pipeline
+  // one allocation for all pipelines: a power of two of at least 32 columns
+  static constexpr int kTmemAlloc = kP * kTmemCols <= 32 ? 32 : kP * kTmemCols <= 64 ? 64
+                                    : kP * kTmemCols <= 128 ? 128 : kP * kTmemCols <= 256 ? 256 : 512;
+  static_assert(kP * kTmemCols <= 512, "TMEM budget");
+  static_assert(kStageBytes % 1024 == 0 && kSubBytes % 1024 == 0, "128-byte swizzled stages need 1024-byte alignment");
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
 };
@@ -268,30 +288,39 @@ __device__ __forceinline__ void store_row16(const GemmArgs& p, int row, int col,
     if (col + j < p.Nk) store_out(p, base + j, v[j]);
 }
 
+// Named barrier among the 128 epilogue threads of one pipeline.
+__device__ __forceinline__ void epi_sync(int sub) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + sub) : "memory");
+}
+
 template <int BN, bool MX, int ACC>
-__global__ void __launch_bounds__(192, ctas_per_sm<BN>())
+__global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmArgs p) {
   using C = Cfg<BN, MX, ACC>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint32_t s_tmem_base;
+  const int sub = threadIdx.x / 192;  // pipeline of this thread
+  const int lt = threadIdx.x % 192;
+  const int warp = lt >> 5, lane = lt & 31;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023)) +
+                  sub * C::kSubBytes;
   uint8_t* misc = smem + S * C::kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;
   uint64_t* acc_empty = acc_full + ACC;
   uint64_t* drain = acc_empty + ACC;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(drain + 1);
   volatile int* s_epi_fail = s_abort + 1;
+  volatile int* s_last = s_abort + 2;  // stream-K: this pipeline completes the current tile
   int* s_mt = reinterpret_cast<int*>(misc + 1024);
   int* s_off = s_mt + (kMaxGroups + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vb = blockIdx.x * C::kP + sub, vg = gridDim.x * C::kP;
 
   // prologue (overlaps the tail of the previous kernel under programmatic launch)
-  if (threadIdx.x == 0) {
+  if (lt == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -303,17 +332,18 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
     mbar_init(drain, 1);
     *s_abort = 0;
     *s_epi_fail = 0;
+    *s_last = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) {
-    tmem_alloc(s_tmem, C::kTmemCols);
+  if (sub == 0 && warp == 1) {  // one allocation for all pipelines of the CTA
+    tmem_alloc(&s_tmem_base, C::kTmemAlloc);
     tmem_relinquish();
   }
-  // the finalize kernel (if any) may launch now and wait for this grid to complete
+  // the next kernel on the stream may launch now; it waits for this grid to complete
   allow_dependents();
   if (p.mode == kModeGrouped && warp == 2) {
     wait_prior_grids();  // the offsets may come from the previous kernel
@@ -345,7 +375,7 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *s_tmem;
+  const uint32_t tmem = s_tmem_base + sub * C::kTmemCols;
   const uint32_t sf_col0 = ACC * BN;
 
   if (warp == 0) {
@@ -392,7 +422,7 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
       bool replayed = !early;
       auto replay = [&]() {
         wait_prior_grids();
-        Sched<BN> rs(p, s_mt, s_off);
+        Sched<BN> rs(p, s_mt, s_off, vb, vg);
         Work rw;
         int j = 0;
         while (j < npend && rs.next(rw))
@@ -400,7 +430,7 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
         replayed = true;
       };
       if (!early) wait_prior_grids();
-      Sched<BN> sch(p, s_mt, s_off);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg);
       Work w;
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
@@ -440,7 +470,7 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      Sched<BN> sch(p, s_mt, s_off);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
       int stage = 0, iter = 0;
@@ -506,11 +536,13 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-      const int rl = q * 32 + lane;     // accumulator row (TMEM lane) of this thread
+    // a warp reads the TMEM lane quarter given by its warp index in the CTA, modulo 4
+    const int q = (threadIdx.x >> 5) & 3;
+    const int rl = q * 32 + lane;     // accumulator row (TMEM lane) of this thread
+    const int et = lt - 64;           // 0..127
     wait_prior_grids();               // the global scales come from earlier kernels
     const float ga = p.ga ? *p.ga : 1.0f;
-    Sched<BN> sch(p, s_mt, s_off);
+    Sched<BN> sch(p, s_mt, s_off, vb, vg);
     Work w;
     int iter = 0;
     while (sch.next(w)) {
@@ -518,11 +550,11 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
       const uint32_t par = (iter / ACC) & 1;
       // the four epilogue warps decide together whether to go on, so that none of them
       // is left behind at a named barrier
-      if (lane == 0 && !mbar_wait(&acc_full[acc], par, s_abort)) {
+      if (et == 0 && !mbar_wait(&acc_full[acc], par, s_abort)) {
         latch_timeout(s_abort, p.status);
         *s_epi_fail = 1;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      epi_sync(sub);
       if (*s_epi_fail) break;
       tc_fence_after();
       const float gb = p.gb ? p.gb[w.group] : 1.0f;
@@ -560,48 +592,62 @@ __global__ void __launch_bounds__(192, ctas_per_sm<BN>())
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       ++iter;
+      if (p.mode == kModeStreamK) {
+        // The pipeline whose partial sums complete the tile's K range writes the tile:
+        // every pipeline publishes its reductions (fence), then adds the K steps it
+        // covered to the tile's counter; the one that brings it to num_kb reads the
+        // sums back from L2, scales, converts, stores, and clears sums and counter.
+        __threadfence();
+        epi_sync(sub);
+        if (et == 0) {
+          __threadfence();
+          const int covered = w.kb1 - w.kb0;
+          const int before = atomicAdd(p.tile_cnt + w.tile, covered);
+          *s_last = before + covered == p.num_kb ? 1 : 0;
+        }
+        epi_sync(sub);
+        if (*s_last) {
+          __threadfence();
+          if (row_ok) {
+            float* src = p.ws + static_cast<int64_t>(row) * p.Nk;
+            for (int c = 0; c < BN; c += 16) {
+              const int col = w.n0 + c;
+              if (col >= p.Nk) break;
+              float v[16];
+              if ((p.Nk & 3) == 0 && col + 16 <= p.Nk) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                  const float4 t = __ldcg(reinterpret_cast<const float4*>(src + col + j));
+                  __stcg(reinterpret_cast<float4*>(src + col + j), make_float4(0.f, 0.f, 0.f, 0.f));
+                  v[j] = t.x * scale;
+                  v[j + 1] = t.y * scale;
+                  v[j + 2] = t.z * scale;
+                  v[j + 3] = t.w * scale;
+                }
+              } else {
+                for (int j = 0; j < 16; ++j) {
+                  v[j] = 0.0f;
+                  if (col + j < p.Nk) {
+                    v[j] = __ldcg(src + col + j) * scale;
+                    __stcg(src + col + j, 0.0f);
+                  }
+                }
+              }
+              store_row16(p, row, col, v);
+            }
+          }
+          if (et == 0) p.tile_cnt[w.tile] = 0;
+        }
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
+  if (sub == 0 && warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
-}
-
-// Stream-K finalize: D = gA * gB * workspace (kernel orientation [Mk, Nk], written back
-// transposed when the operands were swapped), then the workspace is cleared for the next
-// call.  Launched right after the GEMM with programmatic dependent launch.
-__global__ void __launch_bounds__(256) splitk_finalize_kernel(const GemmArgs p) {
-  allow_dependents();  // the next kernel may launch; it waits for this grid before using D
-  wait_prior_grids();
-  const float scale = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f);
-  const int nq = (p.Nk + 3) / 4;
-  const int64_t total = static_cast<int64_t>(p.Mk) * nq;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    // consecutive threads take consecutive kernel rows: the transposed stores coalesce
-    const int r = static_cast<int>(idx % p.Mk);
-    const int c = static_cast<int>(idx / p.Mk) * 4;
-    float* src = p.ws + static_cast<int64_t>(r) * p.Nk + c;
-    float v[4];
-    if ((p.Nk & 3) == 0) {
-      const float4 t = __ldcs(reinterpret_cast<const float4*>(src));
-      *reinterpret_cast<float4*>(src) = make_float4(0.f, 0.f, 0.f, 0.f);
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    } else {
-      for (int j = 0; j < 4; ++j) {
-        v[j] = c + j < p.Nk ? src[j] : 0.0f;
-        if (c + j < p.Nk) src[j] = 0.0f;
-      }
-    }
-    for (int j = 0; j < 4 && c + j < p.Nk; ++j) {
-      const int64_t o = p.transposed ? static_cast<int64_t>(c + j) * p.ldo + r : static_cast<int64_t>(r) * p.ldo + c + j;
-      store_out(p, o, v[j] * scale);
-    }
+    tmem_dealloc(s_tmem_base, C::kTmemAlloc);
   }
 }
 
@@ -646,7 +692,7 @@ struct MapCacheEntry {
   uint32_t box;
   CUtensorMap map;
 };
-static bool make_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+bool make_tensor_map_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
   constexpr int kEntries = 32;
   static MapCacheEntry cache[kEntries];
   static int used = 0, next = 0;
@@ -719,7 +765,7 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
   if (tiles < 2 * sms && pl.num_kb >= 4) {
     pl.mode = kModeStreamK;
     pl.units = tiles * pl.num_kb;
-    pl.ws_bytes = static_cast<size_t>(M * N) * 4;
+    pl.ws_bytes = (static_cast<size_t>(M * N) * 4 + 255) / 256 * 256 + (static_cast<size_t>(tiles) * 4 + 255) / 256 * 256;
   } else {
     pl.mode = kModeTile;
     pl.units = tiles;
@@ -728,7 +774,15 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
   return pl;
 }
 
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx) { return make_plan(M, N, K, 0, mx).ws_bytes; }
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx) {
+  if (!mx && decode_eligible(M, N, K)) return decode_workspace_bytes(M, N);
+  return make_plan(M, N, K, 0, mx).ws_bytes;
+}
+
+// the quantize workspace (tensor amax), then the GEMM's
+size_t gemm_bf16a_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return (kQuantWorkspaceBytes + 255) / 256 * 256 + gemm_workspace_bytes(M, N, K, 0);
+}
 
 template <int BN, bool MX, int ACC>
 static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid, cudaStream_t st) {
@@ -744,12 +798,12 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_done[dev] = true;
   }
-  // programmatic dependent launch: the prologue (barriers, TMEM, descriptor prefetch)
-  // overlaps the previous kernel on the stream; the kernel waits for it before reading
-  // any global memory
+  // programmatic dependent launch: the prologue (barriers, TMEM, descriptor prefetch,
+  // and loads of an operand the caller marked as ready) overlaps the previous kernel on
+  // the stream; everything else waits for it
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid * C::kCtasPerSm);
-  cfg.blockDim = dim3(192);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -757,30 +811,47 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
-  if (e != cudaSuccess || a.mode != kModeStreamK) return e;
-  cudaLaunchConfig_t fin = cfg;
-  const int64_t work = static_cast<int64_t>(a.Mk) * ((a.Nk + 3) / 4);
-  fin.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * num_sms()))));
-  fin.blockDim = dim3(256);
-  fin.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&fin, splitk_finalize_kernel, a);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
 }
 
 template <bool MX>
-static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid,
+static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
                             cudaStream_t st) {
+  // one CTA per SM at most; a CTA holds pipes_per_cta<BN>() pipelines
+  auto grid_for = [&](int pipes) {
+    if (pl.mode == kModeGrouped) return num_sms();
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((pl.units + pipes - 1) / pipes, num_sms())));
+  };
   switch (pl.BN) {
-    case 16: return run<16, MX, 2>(ta, tb, a, grid, st);
-    case 32: return run<32, MX, 2>(ta, tb, a, grid, st);
-    case 64: return run<64, MX, 2>(ta, tb, a, grid, st);
-    case 128: return run<128, MX, 2>(ta, tb, a, grid, st);
-    default: return run<256, MX, 1>(ta, tb, a, grid, st);
+    case 16: return run<16, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<16>()), st);
+    case 32: return run<32, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<32>()), st);
+    case 64: return run<64, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<64>()), st);
+    case 128: return run<128, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<128>()), st);
+    default: return run<256, MX, 1>(ta, tb, a, grid_for(pipes_per_cta<256>()), st);
   }
 }
 
 int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err) {
   const int grouped = g.num_groups > 0;
+  if (!grouped && !g.mx && decode_eligible(g.M, g.N, g.K)) {
+    // a few activation rows: the decode kernel (the weights are problem B)
+    DecodeProblem q{};
+    q.W = g.B;
+    q.sW = g.sB;
+    q.gW = g.gB;
+    q.Xq = g.A;
+    q.Xs = g.sA;
+    q.gX = g.gA;
+    q.M = g.M;
+    q.N = g.N;
+    q.K = g.K;
+    q.D = g.D;
+    q.out_bf16 = g.out_bf16;
+    q.ws = g.ws;
+    q.ws_bytes = g.ws_bytes;
+    q.weights_ready = g.weights_ready;
+    return launch_decode(q, status, st, why, err);
+  }
   const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx);
   if (g.ws_bytes < pl.ws_bytes || (pl.ws_bytes && !g.ws)) {
     *why = "workspace too small (see fp4_gemm_workspace_size)";
@@ -798,8 +869,8 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
     std::swap(rowsA, rowsB);
   }
   CUtensorMap ta, tb;
-  if (!make_map(&ta, kA, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsA), 128) ||
-      !make_map(&tb, kB, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsB), static_cast<uint32_t>(pl.BN))) {
+  if (!make_tensor_map_u8(&ta, kA, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsA), 128) ||
+      !make_tensor_map_u8(&tb, kB, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsB), static_cast<uint32_t>(pl.BN))) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
     return 1;
   }
@@ -831,6 +902,7 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   a.status = status;
   if (pl.mode == kModeStreamK) {
     a.ws = static_cast<float*>(g.ws);
+    a.tile_cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(g.ws) + (static_cast<size_t>(g.M * g.N) * 4 + 255) / 256 * 256);
   }
   if (grouped) {
     a.num_groups = g.num_groups;
@@ -841,13 +913,7 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   } else {
     a.sfb_rbs = static_cast<int>((rowsB + 127) / 128);
   }
-  // CTAs per SM are applied by run(); a tile schedule never launches more CTAs than units
-  int grid;
-  const int per_sm = pl.BN <= 64 ? 2 : 1;
-  if (pl.mode == kModeGrouped) grid = num_sms();
-  else grid = static_cast<int>(std::min<int64_t>((pl.units + per_sm - 1) / per_sm, num_sms()));
-  grid = std::max(grid, 1);
-  const cudaError_t e = g.mx ? dispatch<true>(pl, ta, tb, a, grid, st) : dispatch<false>(pl, ta, tb, a, grid, st);
+  const cudaError_t e = g.mx ? dispatch<true>(pl, ta, tb, a, st) : dispatch<false>(pl, ta, tb, a, st);
   if (e != cudaSuccess) {
     *err = e;
     return 2;

@@ -1,6 +1,7 @@
 // fp4_internal.h -- declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <algorithm>
 #include <cstdint>
@@ -26,6 +27,13 @@ cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float*
 cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
                                uint8_t* scales, const float* g, const int32_t* offsets, int num_groups,
                                unsigned* status, cudaStream_t st);
+// Small tensors (see quantize_small_fits): amax, global scale and 1-D quantize in one
+// launch of one thread-block cluster; the scale buffer is zero-filled and written.
+constexpr int kSmallCtas = 8, kSmallThreads = 512;
+bool quantize_small_fits(int64_t rows, int64_t cols, int bf16, int mx);
+cudaError_t launch_quantize_small(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
+                                  uint8_t* scales, const float* g_in, float* g_out, unsigned* status,
+                                  cudaStream_t st);
 cudaError_t launch_quantize_2d(const void* x, int64_t rows, int64_t cols, int bf16, uint8_t* codes,
                                uint8_t* scales, uint8_t* codesT, uint8_t* scalesT, const float* g,
                                unsigned* status, cudaStream_t st);
@@ -51,6 +59,34 @@ struct GemmProblem {
 };
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx);
+
+size_t gemm_bf16a_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+// Encoded 2-D TMA map of a [rows, inner_bytes] uint8 matrix, boxes of box_rows x 128
+// bytes with the 128-byte swizzle (cached per address and shape).
+bool make_tensor_map_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows);
+
+// Decode-shaped NVFP4 GEMM (1 <= M <= 32): D [M, N] = gX gW (X_hat . W_hat^T), with the
+// activations either pre-quantized (Xq / Xs / gX) or BF16 (X, quantized inside the
+// kernel into Xq_out / Xs_out / gX_out).
+struct DecodeProblem {
+  const uint8_t *W, *sW;
+  const float* gW;
+  const uint8_t *Xq, *Xs;
+  const float* gX;
+  const void* X;
+  uint8_t *Xq_out, *Xs_out;
+  float* gX_out;
+  int64_t M, N, K;
+  void* D;
+  int out_bf16;
+  void* ws;
+  size_t ws_bytes;
+  int weights_ready;
+};
+bool decode_eligible(int64_t M, int64_t N, int64_t K);
+size_t decode_workspace_bytes(int64_t M, int64_t N);
+int launch_decode(const DecodeProblem& q, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err);
 // Returns 0 on success, 1 on an unsupported shape / too-small workspace (message in
 // *why), or 2 on a CUDA error (code in *err).
 int launch_gemm(const GemmProblem& p, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err);

@@ -284,10 +284,7 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
         sb = e8m0_code(__fdiv_rn(amax_b, 6.0f));
         mul = e8m0_inverse(sb);
       } else {
-        const float t = __fdiv_rn(amax_b, 6.0f);
-        sb = e4m3_code(__fdiv_rn(t, g));
-        const float denom = __fmul_rn(e4m3_value(sb), g);
-        mul = denom == 0.0f ? 0.0f : __frcp_rn(denom);
+        mul = nvfp4_block_scale(amax_b, g, sb);
       }
       float s[EPC];
 #pragma unroll
@@ -317,6 +314,148 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
     __syncthreads();
   }
   if (bad) atomicOr(p.status, kStatusNonFinite);
+}
+
+// ------------------------------------------------------------------ small tensors
+// A tensor of at most kSmallThreads * kSmallCtas * NB blocks (e.g. 32 x 8192 BF16
+// activations of a decode step) is quantized by one thread-block cluster in a single
+// launch: every thread loads its NB blocks into registers, the cluster combines the
+// tensor amax through distributed shared memory, and the registers are encoded -- one
+// read of x, and no second kernel waiting for the amax.
+struct SmallArgs {
+  const void* x;
+  int64_t rows, cols;
+  uint8_t* codes;
+  uint8_t* scales;
+  int64_t scale_bytes;  // padded size of the scale buffer (zero-filled by the kernel)
+  const float* g_in;    // NVFP4: caller's global scale, or null to compute it
+  float* g_out;         // may be null
+  unsigned* status;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Store v into the shared-memory word at local address `local` of cluster CTA `rank`.
+__device__ __forceinline__ void st_cluster_u32(const void* local, uint32_t rank, uint32_t v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <typename T, int BLOCK>
+struct SmallCfg {
+  static constexpr int kChunks = BLOCK * static_cast<int>(sizeof(T)) / 16;  // 16-byte loads per block
+  static constexpr int kNB = 8 / kChunks;                                    // blocks per thread
+};
+
+template <typename T, int BLOCK, bool MX, bool HW>
+__global__ void __cluster_dims__(kSmallCtas, 1, 1) __launch_bounds__(kSmallThreads)
+    quantize_small_kernel(const SmallArgs p) {
+  using SC = SmallCfg<T, BLOCK>;
+  constexpr int CH = SC::kChunks, NB = SC::kNB, EPC = Elem<T>::kPerChunk;
+  constexpr int TT = kSmallThreads * kSmallCtas;
+  __shared__ uint32_t s_warp[kSmallThreads / 32];
+  __shared__ uint32_t s_cta[kSmallCtas];
+
+  allow_dependents();
+  wait_prior_grids();  // x may come from the kernel just before; codes / scales may still be read by it
+  const uint32_t rank = cluster_rank();
+  const int gt = static_cast<int>(rank) * kSmallThreads + threadIdx.x;
+  // zero-fill the padded scale buffer; the cluster barrier below orders these stores
+  // before the scale bytes written after it
+  for (int64_t o = static_cast<int64_t>(gt) * 16; o < p.scale_bytes; o += static_cast<int64_t>(TT) * 16)
+    *reinterpret_cast<uint4*>(p.scales + o) = make_uint4(0, 0, 0, 0);
+
+  const int64_t bpr = p.cols / BLOCK;  // blocks per row
+  const int64_t nblocks = p.rows * bpr;
+  uint4 u[NB][CH];
+  uint32_t bm[NB];
+  uint32_t tmax = 0;
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    const int64_t b = gt + static_cast<int64_t>(i) * TT;
+    const uint8_t* src = static_cast<const uint8_t*>(p.x) + b * BLOCK * static_cast<int64_t>(sizeof(T));
+#pragma unroll
+    for (int j = 0; j < CH; ++j) u[i][j] = b < nblocks ? ld_stream(src + j * 16) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      float v[EPC];
+      Elem<T>::unpack(u[i][j], v);
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) m = max(m, abs_bits(v[e]));
+    }
+    bm[i] = m;
+    tmax = max(tmax, m);
+  }
+  // tensor amax: warp -> CTA -> every CTA of the cluster
+  tmax = __reduce_max_sync(0xFFFFFFFFu, tmax);
+  if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = tmax;
+  __syncthreads();
+  if (threadIdx.x < kSmallCtas) {
+    uint32_t cm = 0;
+    for (int w = 0; w < kSmallThreads / 32; ++w) cm = max(cm, s_warp[w]);
+    st_cluster_u32(&s_cta[rank], threadIdx.x, cm);  // thread t delivers this CTA's max to CTA t
+  }
+  cluster_sync_all();
+  uint32_t am = 0;
+#pragma unroll
+  for (int c = 0; c < kSmallCtas; ++c) am = max(am, s_cta[c]);
+  float g = 1.0f;
+  if constexpr (!MX) {
+    const float amax = __uint_as_float(am);
+    g = p.g_in ? *p.g_in : (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f);  // 2688 = 6 * 448
+  }
+  if (gt == 0 && p.g_out) *p.g_out = g;
+  if (gt == 0 && am >= 0x7F800000u) atomicOr(p.status, kStatusNonFinite);
+
+  const int64_t spad = ((bpr + 3) / 4) * 4;  // scale columns padded to whole atoms
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    const int64_t b = gt + static_cast<int64_t>(i) * TT;
+    if (b >= nblocks) continue;
+    const int64_t r = b / bpr, c = b % bpr;
+    uint32_t sb;
+    float mul;
+    if constexpr (MX) {
+      sb = e8m0_code(__fdiv_rn(__uint_as_float(bm[i]), 6.0f));
+      mul = e8m0_inverse(sb);
+    } else {
+      mul = nvfp4_block_scale(__uint_as_float(bm[i]), g, sb);
+    }
+    uint32_t packed[BLOCK / 8];
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      float v[EPC];
+      Elem<T>::unpack(u[i][j], v);
+      float s[EPC];
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) s[e] = (!MX && v[e] == 0.0f) ? v[e] : __fmul_rn(v[e], mul);
+      if constexpr (EPC == 8) {
+        packed[j] = pack8<HW>(s);
+      } else {
+        const uint32_t h = pack4<HW>(s);
+        if (j & 1) packed[j / 2] |= h << 16;
+        else packed[j / 2] = h;
+      }
+    }
+    uint8_t* dst = p.codes + b * (BLOCK / 2);
+    if constexpr (BLOCK == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    else *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    p.scales[((r / 128) * (spad / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4] =
+        static_cast<uint8_t>(sb);
+  }
 }
 
 // x * (1/denom) with a zero element kept zero when the reciprocal overflowed.
@@ -379,12 +518,9 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
     m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     bad |= m >= 0x7F800000u;
     if (sub == 0) {
-      const float amax_b = __uint_as_float(m);
-      const float t = __fdiv_rn(amax_b, 6.0f);
-      const uint32_t sb = e4m3_code(__fdiv_rn(t, g));
-      const float denom = __fmul_rn(e4m3_value(sb), g);
+      uint32_t sb;
+      s_mul[pr][pc] = nvfp4_block_scale(__uint_as_float(m), g, sb);
       s_sb[pr][pc] = static_cast<uint8_t>(sb);
-      s_mul[pr][pc] = denom == 0.0f ? 0.0f : __frcp_rn(denom);
     }
   }
   __syncthreads();
@@ -549,6 +685,49 @@ cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf
   a.status = status;
   if (bf16) return mx ? launch_q1d_t<__nv_bfloat16, 32, true>(a, st) : launch_q1d_t<__nv_bfloat16, 16, false>(a, st);
   return mx ? launch_q1d_t<float, 32, true>(a, st) : launch_q1d_t<float, 16, false>(a, st);
+}
+
+template <typename T, int BLOCK>
+static constexpr int64_t small_capacity_blocks() {
+  return static_cast<int64_t>(kSmallThreads) * kSmallCtas * SmallCfg<T, BLOCK>::kNB;
+}
+
+bool quantize_small_fits(int64_t rows, int64_t cols, int bf16, int mx) {
+  const int64_t nb = rows * (cols / (mx ? 32 : 16));
+  if (bf16) return nb <= (mx ? small_capacity_blocks<__nv_bfloat16, 32>() : small_capacity_blocks<__nv_bfloat16, 16>());
+  return nb <= (mx ? small_capacity_blocks<float, 32>() : small_capacity_blocks<float, 16>());
+}
+
+template <typename T, int BLOCK, bool MX>
+static cudaError_t launch_small_t(const SmallArgs& a, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSmallCtas);  // one cluster (its size is fixed by the kernel)
+  cfg.blockDim = dim3(kSmallThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_small_kernel<T, BLOCK, MX, kE2M1Hardware>, a);
+}
+
+cudaError_t launch_quantize_small(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
+                                  uint8_t* scales, const float* g_in, float* g_out, unsigned* status,
+                                  cudaStream_t st) {
+  SmallArgs a;
+  a.x = x;
+  a.rows = rows;
+  a.cols = cols;
+  a.codes = codes;
+  a.scales = scales;
+  const int64_t scols = cols / (mx ? 32 : 16);
+  a.scale_bytes = ((rows + 127) / 128) * 128 * (((scols + 3) / 4) * 4);
+  a.g_in = g_in;
+  a.g_out = g_out;
+  a.status = status;
+  if (bf16) return mx ? launch_small_t<__nv_bfloat16, 32, true>(a, st) : launch_small_t<__nv_bfloat16, 16, false>(a, st);
+  return mx ? launch_small_t<float, 32, true>(a, st) : launch_small_t<float, 16, false>(a, st);
 }
 
 cudaError_t launch_quantize_2d(const void* x, int64_t rows, int64_t cols, int bf16, uint8_t* codes,

@@ -128,7 +128,8 @@ fp4_status fp4_dequantize(const uint8_t* codes_dev, const uint8_t* scales_dev,
                           float* out_dev, void* stream);
 
 /* Device workspace bytes fp4_gemm needs for this shape (0 if none).  It must be
- * zero-filled before first use; every call leaves it zero-filled again. */
+ * zero-filled before first use; every call leaves it zero-filled again.  After a call
+ * that latched FP4_ERR_TIMEOUT its contents are undefined: zero it again. */
 size_t fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt);
 
 /* Block-scaled FP4 GEMM on the 5th-generation tensor cores ("Rubin FP4 GEMM overview"
@@ -157,6 +158,28 @@ fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev,
                        const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
                        int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,
                        void* workspace_dev, size_t workspace_bytes, unsigned flags, void* stream);
+
+/* BF16-activation GEMM (quantize-on-load): D = gX * gB * (Xq . Bq^T) where Xq is the
+ * NVFP4 quantization of the bf16 activations X [M, K] (tensor amax -> gX, 16-blocks,
+ * exactly as fp4_quantize) and B [N, K] holds pre-quantized NVFP4 weights.  The
+ * activations' codes [M, K/2], scales (fp4_scales_bytes(M, K, NVFP4)) and gX are
+ * written to Xcodes_dev / Xscales_dev / gX_dev as well.  ("Rubin FP4 GEMM overview"
+ * 3.2: loads feed the tensor cores; the activations enter in BF16.)
+ *   M <= 32 (decode): one cooperative launch.  Every CTA reduces a share of X, the
+ *     shares meet through per-CTA slots in the workspace (bounded waits), and each CTA
+ *     quantizes the K segment of X it needs straight into shared memory while its
+ *     first weight stages stream in; split-K partial sums are reduced in the workspace
+ *     and written out by the CTA that owns each tile.
+ *   M > 32: fp4_quantize then fp4_gemm_ex, chained with programmatic dependent launch.
+ * flags: FP4_GEMM_WEIGHTS_READY as for fp4_gemm_ex.  workspace: at least
+ * fp4_gemm_bf16a_workspace_size(M, N, K) bytes, zero-filled before its first use; the
+ * library keeps its contents consistent from call to call, so do not modify it between
+ * calls, and calls sharing one workspace must not overlap. */
+size_t fp4_gemm_bf16a_workspace_size(int64_t M, int64_t N, int64_t K);
+fp4_status fp4_gemm_bf16a(const void* X_dev, const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
+                          int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,
+                          uint8_t* Xcodes_dev, uint8_t* Xscales_dev, float* gX_dev,
+                          void* workspace_dev, size_t workspace_bytes, unsigned flags, void* stream);
 
 /* fp4_gemm for callers that cannot allocate device memory.  The pages have no
  * counterpart to this entry point: it exists for code that runs while a CUDA graph is

@@ -147,6 +147,23 @@ def test_gemm_repeatable_and_workspace_clean():
         check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4))
 
 
+def test_split_k_counters_reset_between_shapes():
+    """The split-over-K path counts each tile's finished K steps in the workspace; the
+    pipeline completing a tile writes it and resets its counter, so calls of different
+    shapes can share one workspace back to back."""
+    shapes = [(16, 1024, 4096), (1, 256, 512), (32, 640, 2048), (16, 1024, 4096)]
+    ws = fp4.Workspace()
+    for i, (m, n, k) in enumerate(shapes):
+        xa = random_input(m, k, 40 + i, torch.bfloat16)
+        xb = random_input(n, k, 50 + i, torch.float32, std=0.02)
+        qa, qb = gpu_quantize(xa.cuda(), fp4.NVFP4, 16), gpu_quantize(xb.cuda(), fp4.NVFP4, 16)
+        d = fp4.gemm(qa, qb, torch.bfloat16, workspace=ws)
+        torch.cuda.synchronize()
+        assert not ws.buf.any(), f"workspace not clean after {m}x{n}x{k}"
+        oa, ob = oracle_quantize(xa, fp4.NVFP4, 16), oracle_quantize(xb, fp4.NVFP4, 16)
+        check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label=f"{m}x{n}x{k}")
+
+
 def test_grouped_gemm_moe_small():
     """Grouped MXFP4 GEMM with an empty expert and ragged expert sizes."""
     offsets = np.array([0, 130, 130, 300, 301, 560], np.int32)
@@ -212,3 +229,55 @@ def test_gemm_ex_weights_ready_decode():
         assert fp4.fp4_get_status() == fp4.OK
         oa = oracle_quantize(xa, fp4.NVFP4, 16)
         check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label=f"rep {rep}")
+
+
+def _bf16a(xa, qb, n, k, out_dtype=torch.bfloat16, flags=0, ws=None):
+    m = xa.shape[0]
+    dev = "cuda"
+    xq = torch.empty(m, k // 2, dtype=torch.uint8, device=dev)
+    xs = torch.empty(fp4.fp4_scales_bytes(m, k, fp4.NVFP4), dtype=torch.uint8, device=dev)
+    gx = torch.empty(1, dtype=torch.float32, device=dev)
+    d = torch.empty(m, n, dtype=out_dtype, device=dev)
+    if ws is None:
+        ws = torch.zeros(fp4.fp4_gemm_bf16a_workspace_size(m, n, k), dtype=torch.uint8, device=dev)
+    fp4.fp4_gemm_bf16a(xa, qb.codes, qb.scales, qb.g, m, n, k, d, fp4.BF16 if out_dtype == torch.bfloat16 else fp4.F32,
+                       xq, xs, gx, ws, ws.numel(), flags)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_status() == fp4.OK
+    return d, fp4.Quantized(xq, xs, gx, m, k, fp4.NVFP4), ws
+
+
+@pytest.mark.parametrize("m,n,k,flags", [(16, 1024, 4096, 0), (16, 1024, 4096, 1), (1, 256, 256, 0),
+                                         (32, 512, 2048, 1), (5, 384, 96, 0), (200, 256, 512, 1)])
+def test_gemm_bf16a_matches_oracle(m, n, k, flags):
+    """Activations quantized inside the call: codes, scales and g bit-exact; D in tolerance."""
+    from fp4_testutil import assert_quant_equal
+    xa = random_input(m, k, 300 + m, torch.bfloat16).cuda()
+    xb = random_input(n, k, 301 + n, torch.float32, std=0.02, outliers=False)
+    qb = gpu_quantize(xb.cuda(), fp4.NVFP4, 16)
+    ob = oracle_quantize(xb, fp4.NVFP4, 16)
+    ws = None
+    for rep in range(2):   # the workspace carries state from call to call
+        d, qx, ws = _bf16a(xa, qb, n, k, flags=flags, ws=ws)
+        ox = oracle_quantize(xa.cpu(), fp4.NVFP4, 16)
+        assert_quant_equal(qx, ox, f"activations {m}x{k} rep {rep}")
+        check_gemm(d, dequant_oracle(ox, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label=f"{m}x{n}x{k} rep {rep}")
+
+
+def test_gemm_bf16a_full_decode_shape_sampled():
+    """The decode configuration in the bench's launch shape (16 x 28672 x 8192)."""
+    x, w = workloads.decode_inputs()
+    qb = gpu_quantize(w.cuda(), fp4.NVFP4, 16)
+    d, qx, _ = _bf16a(x.cuda(), qb, 28672, 8192, flags=fp4.GEMM_WEIGHTS_READY)
+    from fp4_testutil import assert_quant_equal, host_input
+    ox = oracle_quantize(x, fp4.NVFP4, 16)
+    assert_quant_equal(qx, ox, "decode activations")
+    # sampled weight rows (output columns): quantize them with W's global scale
+    hw = host_input(w)
+    g = oracle.global_scale(oracle.amax(hw))
+    cols = np.unique(np.concatenate([[0, 28671], np.random.default_rng(1).integers(0, 28672, 256)]))
+    ob = oracle.quantize(hw[cols], oracle.NVFP4, 16, g_in=g)
+    b_hat = oracle.dequantize(ob["codes"], ob["scales"], ob["g"])
+    d_ref, s = oracle.gemm_reference(dequant_oracle(ox, fp4.NVFP4), b_hat)
+    got = d[:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - d_ref) <= oracle.gemm_tolerance(d_ref, s, True))

@@ -76,9 +76,11 @@ def test_worked_blocks_on_gpu(idx):
     assert q.scales.cpu().numpy()[0] == scale
 
 
+# (130, 128) runs the single-launch path for small tensors, (300, 1024) the amax +
+# quantize kernels of larger ones
+@pytest.mark.parametrize("rows,cols", [(130, 128), (300, 1024)])
 @pytest.mark.parametrize("kind", ["zeros", "neg_zeros", "tiny", "huge", "constant", "subnormal"])
-def test_quantize_edge_tensors(kind):
-    rows, cols = 130, 128
+def test_quantize_edge_tensors(kind, rows, cols):
     if kind == "zeros":
         x = torch.zeros(rows, cols)
     elif kind == "neg_zeros":
@@ -104,9 +106,10 @@ def test_quantize_block_far_below_tensor_amax():
     assert_quant_equal(gq, oracle_quantize(x, fp4.NVFP4, 16))
 
 
+@pytest.mark.parametrize("shape", [(64, 64), (400, 1024)])
 @pytest.mark.parametrize("bad", [float("nan"), float("inf"), float("-inf")])
-def test_nonfinite_input_latches_status(bad):
-    x = torch.ones(64, 64)
+def test_nonfinite_input_latches_status(bad, shape):
+    x = torch.ones(*shape)
     x[17, 5] = bad
     fp4.fp4_get_status()
     fp4.quantize(x.cuda(), fp4.NVFP4, 16)
