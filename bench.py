@@ -330,6 +330,241 @@ def run_decode(args, dist: Dist, dev):
     return res
 
 
+# ---------------------------------------------------------------- other workloads
+FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+
+
+def _events_ms(fn, iters: int, warmup: int) -> float:
+    """Average device ms per call of fn(i), events around a batch on the current stream."""
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(iters):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def _check(fp4):
+    if fp4.fp4_get_status() != fp4.OK:
+        raise RuntimeError("device status latched an error")
+
+
+def _copies(per_copy_bytes: int) -> int:
+    """Rotating copies so that one pass over them exceeds the L2 three times."""
+    return max(1, int(np.ceil(3 * L2_BYTES / max(per_copy_bytes, 1))))
+
+
+def _line(workload: str, value, unit: str, ms: float, args, extra: dict) -> dict:
+    res = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "data": "synthetic (seeded, see DESIGN.md)", "config": {"workload": workload}}
+    res.update(extra)
+    return res
+
+
+def run_prefill(args, dev):
+    """Prefill-shaped NVFP4 GEMM 8192^3: BF16 activations quantized every step (tensor amax,
+    then 16-blocks), weights pre-quantized; tensor-bound."""
+    import block_scaled_fp4_04_b200 as fp4
+    m = n = k = 8192
+    x, w = workloads.prefill_inputs(device="cpu")
+    x = x.to(dev)
+    qw = fp4.quantize(w.to(dev), fp4.NVFP4, 16)
+    L = fp4.lib()
+    P = lambda t: t.data_ptr()
+    xc = torch.empty(m, k // 2, dtype=torch.uint8, device=dev)
+    xs = torch.empty(fp4.fp4_scales_bytes(m, k, fp4.NVFP4), dtype=torch.uint8, device=dev)
+    xg = torch.empty(1, dtype=torch.float32, device=dev)
+    wn = fp4.fp4_gemm_bf16a_workspace_size(m, n, k)
+    ws = torch.zeros(wn, dtype=torch.uint8, device=dev)
+    d = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+    sp = torch.cuda.current_stream().cuda_stream
+
+    def step(i):
+        if L.fp4_gemm_bf16a(P(x), P(qw.codes), P(qw.scales), P(qw.g), m, n, k, P(d), fp4.BF16, P(xc), P(xs),
+                            P(xg), P(ws), wn, fp4.GEMM_WEIGHTS_READY, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    def gemm(i):
+        if L.fp4_gemm_ex(fp4.NVFP4, P(xc), P(xs), P(xg), P(qw.codes), P(qw.scales), P(qw.g), m, n, k, P(d),
+                         fp4.BF16, P(ws), wn, 0, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    step_ms = _events_ms(step, args.steps, args.warmup)
+    gemm_ms = _events_ms(gemm, args.steps, args.warmup)
+    _check(fp4)
+    flop = 2.0 * m * n * k
+    hbm, bf16, bf16_s, src = load_peaks()
+    peak = bf16 * FP4_PER_BF16
+    gemm_tf = flop / (gemm_ms * 1e-3) / 1e12
+    step_tf = flop / (step_ms * 1e-3) / 1e12
+    return _line("prefill-shaped NVFP4 GEMM M=N=K=8192, bf16 activations quantized every step, bf16 out",
+                 step_tf, "TFLOP/s", step_ms, args, {
+                     "dtype": "nvfp4 x nvfp4 -> fp32 accumulate, bf16 out",
+                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1>",
+                                  "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tf / peak,
+                                  "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)",
+                                  "frac_of_nominal_9pf": gemm_tf / 9000.0, "launch_ms": gemm_ms,
+                                  "traffic": None},
+                     "step": {"ms": step_ms, "TFLOP/s": step_tf, "contents": "amax + quantize(X) + GEMM"},
+                     "gpu_launches": 3 * args.steps})
+
+
+def run_moe(args, dev):
+    """MXFP4 grouped MoE GEMM: 4096 tokens x top-4 of 32 experts, K=2880, N=5760; the
+    activations are quantized (grouped layout) every step."""
+    import block_scaled_fp4_04_b200 as fp4
+    a, w, offsets, _ = workloads.moe_inputs(device="cpu")
+    E, N, K = w.shape
+    rows = a.shape[0]
+    a = a.to(dev)
+    wq = [fp4.quantize(w[e].to(dev), fp4.MXFP4, 32) for e in range(E)]
+    B = torch.stack([q.codes for q in wq])
+    sB = torch.cat([q.scales for q in wq])
+    del wq
+    off = offsets.to(dev)
+    cap = fp4.fp4_scales_bytes_grouped(rows, E, K, fp4.MXFP4)
+    codes = torch.empty(rows, K // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(cap, dtype=torch.uint8, device=dev)
+    D = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+    L = fp4.lib()
+    P = lambda t: t.data_ptr()
+    sp = torch.cuda.current_stream().cuda_stream
+
+    def quant(i):
+        if L.fp4_quantize_grouped(P(a), rows, K, fp4.BF16, fp4.MXFP4, E, P(off), P(codes), P(scales), None, None,
+                                  None, 0, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    def gemm(i):
+        if L.fp4_gemm_grouped(fp4.MXFP4, E, P(off), P(codes), P(scales), None, P(B), P(sB), None, rows, N, K, P(D),
+                              fp4.BF16, None, 0, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    step_ms = _events_ms(lambda i: (quant(i), gemm(i)), args.steps, args.warmup)
+    gemm_ms = _events_ms(gemm, args.steps, args.warmup)
+    quant_ms = _events_ms(quant, args.steps, args.warmup)
+    _check(fp4)
+    flop = 2.0 * rows * N * K
+    gemm_bytes = E * N * K // 2 + sB.numel() + rows * K // 2 + scales.numel() + rows * N * 2
+    quant_bytes = rows * K * 2 + rows * K // 2 + rows * K // 32
+    hbm, bf16, bf16_s, src = load_peaks()
+    peak = bf16 * FP4_PER_BF16
+    t_roof = max(flop / (peak * 1e12), gemm_bytes / (hbm * 1e9)) * 1e3
+    gemm_tf = flop / (gemm_ms * 1e-3) / 1e12
+    return _line("MXFP4 grouped MoE GEMM: 32 experts, 4096 tokens top-4 (16384 rows), K=2880, N=5760, bf16 out",
+                 flop / (step_ms * 1e-3) / 1e12, "TFLOP/s", step_ms, args, {
+                     "dtype": "mxfp4 x mxfp4 -> fp32 accumulate, bf16 out",
+                     "roofline": {"bound": "tensor" if flop / peak > gemm_bytes / hbm * 1e-3 else "hbm",
+                                  "kernel": "fp4_gemm_kernel<128, mxfp4, 2> (grouped)",
+                                  "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
+                                  "frac": t_roof / gemm_ms,
+                                  "frac_definition": "roofline time (slower of tensor and HBM) / measured time",
+                                  "hbm_GB/s": gemm_bytes / (gemm_ms * 1e-3) / 1e9, "algorithmic_bytes": gemm_bytes,
+                                  "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g}; {src} hbm_gbs",
+                                  "launch_ms": gemm_ms, "traffic": None},
+                     "quantize": {"ms": quant_ms, "GB/s": quant_bytes / (quant_ms * 1e-3) / 1e9,
+                                  "frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / hbm},
+                     "gpu_launches": 2 * args.steps})
+
+
+def run_train(args, dev):
+    """Training-recipe sweep: W quantized once with 16x16 blocks (W and W^T); per step X and
+    dY quantized (16-blocks), forward D = X W^T and backward dX = dY W."""
+    import block_scaled_fp4_04_b200 as fp4
+    hbm, bf16, bf16_s, src = load_peaks()
+    peak = bf16 * FP4_PER_BF16
+    out = []
+    for s in (1024, 2048, 4096, 8192, 16384):
+        x, w, dy = workloads.train_inputs(s, device="cpu")
+        per_copy = 2 * s * s * 2
+        ncopy = _copies(per_copy) if s <= 2048 else 1
+        xs = [x.to(dev) for _ in range(ncopy)]
+        dys = [dy.to(dev) for _ in range(ncopy)]
+        qw = fp4.quantize(w.to(dev), fp4.NVFP4, 256)
+        wt = fp4.transposed(qw)
+        ws = fp4.Workspace(dev)
+        dout = torch.empty(s, s, dtype=torch.bfloat16, device=dev)
+        dxout = torch.empty(s, s, dtype=torch.bfloat16, device=dev)
+        state = {}
+
+        def step(i):
+            qx = fp4.quantize(xs[i % ncopy], fp4.NVFP4, 16, workspace=ws)
+            qd = fp4.quantize(dys[i % ncopy], fp4.NVFP4, 16, workspace=ws)
+            fp4.gemm(qx, qw, out=dout, workspace=ws)
+            fp4.gemm(qd, wt, out=dxout, workspace=ws)
+            state["qx"], state["qd"] = qx, qd
+
+        step_ms = _events_ms(step, max(3, args.steps // 4), args.warmup)
+        qx, qd = state["qx"], state["qd"]
+        fwd_ms = _events_ms(lambda i: fp4.gemm(qx, qw, out=dout, workspace=ws), args.steps, args.warmup)
+        bwd_ms = _events_ms(lambda i: fp4.gemm(qd, wt, out=dxout, workspace=ws), args.steps, args.warmup)
+        _check(fp4)
+        flop = 2.0 * s * s * s
+        out.append({"S": s, "step_ms": step_ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                    "fwd_TFLOP/s": flop / (fwd_ms * 1e-3) / 1e12, "bwd_TFLOP/s": flop / (bwd_ms * 1e-3) / 1e12,
+                    "fwd_frac": flop / (fwd_ms * 1e-3) / 1e12 / peak,
+                    "step_TFLOP/s": 2 * flop / (step_ms * 1e-3) / 1e12,
+                    "l2": f"{ncopy} rotating copies of X, dY" if ncopy > 1 else "inputs larger than L2"})
+        del xs, dys, qw, wt, ws, dout, dxout, state
+        torch.cuda.empty_cache()
+    big = out[-1]
+    return _line("training-recipe sweep M=N=K in {1024..16384}: 2-D NVFP4 W (and W^T) once, X and dY quantized "
+                 "per step, forward X W^T and backward dY W, bf16 out", big["step_TFLOP/s"], "TFLOP/s",
+                 big["step_ms"], args, {
+                     "dtype": "nvfp4 x nvfp4 -> fp32 accumulate, bf16 out",
+                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1> at S=16384",
+                                  "achieved": big["fwd_TFLOP/s"], "peak": peak, "unit": "TFLOP/s",
+                                  "frac": big["fwd_frac"], "traffic": None,
+                                  "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g}"},
+                     "sweep": out, "gpu_launches": None})
+
+
+def run_quantize(args, dev):
+    """Quantize kernels alone: GB/s of algorithmic bytes (NVFP4 reads x twice: amax, encode)."""
+    import block_scaled_fp4_04_b200 as fp4
+    hbm, bf16, bf16_s, src = load_peaks()
+    rows_out = []
+    cases = [
+        ("moe activations bf16 [16384, 2880] -> MXFP4", lambda: workloads.moe_inputs(device="cpu")[0], fp4.MXFP4, 32),
+        ("train X bf16 [16384, 16384] -> NVFP4", lambda: workloads.train_inputs(16384, device="cpu")[0], fp4.NVFP4, 16),
+        ("decode W fp32 [28672, 8192] -> NVFP4", lambda: workloads.decode_inputs(device="cpu")[1], fp4.NVFP4, 16),
+        ("2-D W fp32 [16384, 16384] -> NVFP4 W and W^T", lambda: workloads.train_inputs(16384, device="cpu")[1],
+         fp4.NVFP4, 256),
+    ]
+    for name, make, fmt, blk in cases:
+        x = make().to(dev)
+        rows, cols = x.shape
+        esz = x.element_size()
+        ws = fp4.Workspace(dev)
+        codes = rows * cols // 2
+        sc = fp4.fp4_scales_bytes(rows, cols, fmt)
+        if blk == 256:
+            nbytes = 2 * rows * cols * esz + 2 * (codes + sc)   # amax read + encode read; W and W^T
+        elif fmt == fp4.NVFP4:
+            nbytes = 2 * rows * cols * esz + codes + sc
+        else:
+            nbytes = rows * cols * esz + codes + sc
+        ms = _events_ms(lambda i: fp4.quantize(x, fmt, blk, workspace=ws), max(3, args.steps // 4), args.warmup)
+        _check(fp4)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        rows_out.append({"case": name, "ms": ms, "GB/s": gbs, "frac": gbs / hbm, "bytes": nbytes})
+        del x, ws
+        torch.cuda.empty_cache()
+    best = rows_out[0]
+    return _line("quantize kernels alone (MoE activations, train X, decode W, 2-D W)", best["GB/s"], "GB/s",
+                 best["ms"], args, {
+                     "dtype": "bf16/fp32 in -> nvfp4/mxfp4 codes + scales",
+                     "roofline": {"bound": "hbm", "kernel": "quantize (first case)", "achieved": best["GB/s"],
+                                  "peak": hbm, "unit": "GB/s", "frac": best["frac"], "traffic": None,
+                                  "peak_source": f"{src} hbm_gbs"},
+                     "cases": rows_out, "gpu_launches": None})
+
+
 def cpu_baseline_decode(budget_s: float = 12.0):
     """The oracle, as it stands, on a bounded sample of one decode step: quantize the 16
     activation rows, dequantize a sample of pre-quantized weight rows and take the
@@ -417,7 +652,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "train", "quantize", "all"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -431,6 +666,14 @@ def main():
     dev = torch.device("cuda", dist.local)
     dist.init("nccl")
     try:
+        if args.workload != "decode":
+            if dist.world > 1:
+                raise SystemExit("the additional workloads run on one GPU")
+            names = ["prefill", "moe", "train", "quantize"] if args.workload == "all" else [args.workload]
+            for name in names:
+                print(json.dumps({"prefill": run_prefill, "moe": run_moe, "train": run_train,
+                                  "quantize": run_quantize}[name](args, dev)), flush=True)
+            return
         res = run_decode(args, dist, dev)
         if dist.rank == 0:
             if dist.world == 1 and not args.no_cpu_baseline:

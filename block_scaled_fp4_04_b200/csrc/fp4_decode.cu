@@ -138,6 +138,8 @@ struct DecodeSched {
   }
 };
 
+constexpr int kMaxBatch = 8;
+
 // Weight stages a pipeline of the fused kernel issues before the activations are ready.
 #ifndef FP4_FUSED_PREFILL
 #define FP4_FUSED_PREFILL 2
@@ -157,9 +159,13 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
   uint8_t* s_b = base;                          // activation codes, one swizzled box per K step
   uint8_t* s_bsf = base + C::kBBytes;           // activation scale atoms, 4 per K step
   uint8_t* shared_misc = s_bsf + C::kBSFBytes;
-  uint64_t* b_ready = reinterpret_cast<uint64_t*>(shared_misc);  // activation operand in smem
-  uint64_t* bsf_ready = b_ready + 1;  // [2]: each MMA thread's half of its scales is in TMEM
-  volatile int* s_xfail = reinterpret_cast<volatile int*>(bsf_ready + 2);
+  // The activation operand becomes ready in batches of K steps: b_ready[b] when batch b
+  // is in shared memory, bsf_ready[b] when its scale factors have been copied to TMEM.
+  // Pre-quantized activations arrive in one batch.
+  constexpr int kKpb = FUSED ? 256 / (BN * 8) : C::kMaxSeg;  // K steps per batch
+  uint64_t* b_ready = reinterpret_cast<uint64_t*>(shared_misc);  // [kMaxBatch]
+  uint64_t* bsf_ready = b_ready + kMaxBatch;                     // [kMaxBatch]
+  volatile int* s_xfail = reinterpret_cast<volatile int*>(bsf_ready + kMaxBatch);
 
   const int sub = threadIdx.x / 192, lt = threadIdx.x % 192, warp = lt >> 5, lane = lt & 31;
   uint8_t* ring = base + C::kSharedBytes + sub * C::kSubBytes;
@@ -179,6 +185,8 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
   const int pipe_in_seg = cta_in_seg * C::kP + sub;
   const int kb0 = seg * p.seg_len;
   const int seg_steps = min(p.seg_len, p.num_kb - kb0);
+  const int nbatch = (seg_steps + kKpb - 1) / kKpb;
+  const int seg_atoms = min(seg_steps * 4, p.atoms_k - kb0 * 4);  // activation scale atoms
 
   if (lt == 0) {
     for (int s = 0; s < S; ++s) {
@@ -194,9 +202,10 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
     *s_epi_fail = 0;
     *s_last = 0;
     if (sub == 0) {
-      mbar_init(b_ready, 1);
-      mbar_init(&bsf_ready[0], 1);
-      mbar_init(&bsf_ready[1], 1);
+      for (int b = 0; b < kMaxBatch; ++b) {
+        mbar_init(&b_ready[b], 1);
+        mbar_init(&bsf_ready[b], 1);
+      }
       *s_xfail = 0;
     }
     fence_mbar_init();
@@ -225,10 +234,11 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
       auto load_x = [&]() {
         if (FUSED || sub != 0) return;
         const int atoms = min(seg_steps * 4, p.atoms_k - kb0 * 4);
-        mbar_arrive_expect_tx(b_ready, static_cast<uint32_t>(seg_steps * C::kBBox + atoms * 512));
+        mbar_arrive_expect_tx(&b_ready[0], static_cast<uint32_t>(seg_steps * C::kBBox + atoms * 512));
         const uint64_t pol_x = l2_policy_evict_last();
-        for (int j = 0; j < seg_steps; ++j) tma_load_2d(s_b + j * C::kBBox, &tmX, b_ready, (kb0 + j) * 128, 0, pol_x);
-        bulk_load(s_bsf, p.xs + static_cast<int64_t>(kb0) * 4 * 512, static_cast<uint32_t>(atoms) * 512u, b_ready,
+        for (int j = 0; j < seg_steps; ++j)
+          tma_load_2d(s_b + j * C::kBBox, &tmX, &b_ready[0], (kb0 + j) * 128, 0, pol_x);
+        bulk_load(s_bsf, p.xs + static_cast<int64_t>(kb0) * 4 * 512, static_cast<uint32_t>(atoms) * 512u, &b_ready[0],
                   pol_x);
       };
       if (!p.weights_ready) {
@@ -239,7 +249,7 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
       int tile, k0, k1, stage = 0, issued_n = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
       bool ok = true, x_done = !p.weights_ready;
-      if (FUSED && kFusedPrefill == 0 && !mbar_wait(b_ready, 0, s_abort)) {
+      if (FUSED && kFusedPrefill == 0 && !mbar_wait(&b_ready[0], 0, s_abort)) {
         if (!*s_xfail) d_latch_timeout(s_abort, p.status);
         ok = false;
       }
@@ -269,7 +279,7 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
           // full ring of weight copies
           ++issued_n;
           if (FUSED && issued_n == kFusedPrefill) {
-            if (!mbar_wait(b_ready, 0, s_abort)) {
+            if (!mbar_wait(&b_ready[0], 0, s_abort)) {
               if (!*s_xfail) d_latch_timeout(s_abort, p.status);
               ok = false;
               break;
@@ -298,26 +308,43 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       bool ok = true;
-      // the activations' scale factors go to TMEM once for both pipelines: each MMA
-      // thread copies half of the atoms, commits, and waits for the other half
-      if (!mbar_wait(b_ready, 0, s_abort)) {
+      // The activations' scale factors go to TMEM once for both pipelines, batch by
+      // batch as the operand becomes ready: the first pipeline's MMA thread copies them
+      // (in batch order, as soon as each batch is ready or needed) and commits each batch
+      // to bsf_ready[b]; the second pipeline waits for the batches it needs.
+      int copied = 0, known = 0;
+      const uint32_t bsf_s = smem_u32(s_bsf);
+      auto copy_batch = [&](int b) {
+        tc_fence_after();
+        const int a1 = min((b + 1) * kKpb * 4, seg_atoms);
+        for (int a = b * kKpb * 4; a < a1; ++a) tc_cp_sf_atom(tmem_bsf + a * 4, smem_desc_sf(bsf_s + a * 512));
+        tc_commit(&bsf_ready[b]);
+      };
+      // batches 0..need in TMEM (for this thread's MMAs); false on failure
+      auto ensure = [&](int need) -> bool {
+        if (sub == 0) {
+          while (copied <= need) {
+            if (!mbar_wait(&b_ready[copied], 0, s_abort) || *s_xfail) return false;
+            copy_batch(copied++);
+          }
+          while (copied < nbatch && mbar_try_wait(&b_ready[copied], 0)) {
+            if (*s_xfail) return false;
+            copy_batch(copied++);
+          }
+          return true;  // this thread's own copies precede its MMAs
+        }
+        while (known <= need) {
+          if (!mbar_wait(&bsf_ready[known], 0, s_abort) || *s_xfail) return false;
+          ++known;
+        }
+        tc_fence_after();
+        return true;
+      };
+      auto fail = [&]() {
         if (!*s_xfail) d_latch_timeout(s_abort, p.status);
         ok = false;
-      } else if (*s_xfail) {
-        ok = false;
-      } else {
-        tc_fence_after();
-        const uint32_t sb = smem_u32(s_bsf);
-        const int atoms = min(seg_steps * 4, p.atoms_k - kb0 * 4);
-        const int a0 = sub == 0 ? 0 : atoms / 2, a1 = sub == 0 ? atoms / 2 : atoms;
-        for (int a = a0; a < a1; ++a) tc_cp_sf_atom(tmem_bsf + a * 4, smem_desc_sf(sb + a * 512));
-      }
-      tc_commit(&bsf_ready[sub]);  // also releases the other pipeline when this one failed
-      if (!mbar_wait(&bsf_ready[sub ^ 1], 0, s_abort)) {
-        if (!*s_xfail && ok) d_latch_timeout(s_abort, p.status);
-        ok = false;
-      }
-      tc_fence_after();
+      };
+      if (!ensure(0)) fail();
       DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg);
       const uint32_t ring_s = smem_u32(ring), b_s = smem_u32(s_b);
       int tile, k0, k1, stage = 0, iter = 0;
@@ -334,6 +361,10 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
           if (!mbar_wait(&full[stage], phase, s_abort)) {
             d_latch_timeout(s_abort, p.status);
             ok = false;
+            break;
+          }
+          if (!ensure((kb - kb0) / kKpb)) {
+            fail();
             break;
           }
           tc_fence_after();
@@ -360,6 +391,12 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         if (!ok) break;
         tc_commit(&acc_full[acc]);
         ++iter;
+      }
+      // the other pipeline may still need batches this one did not: copy them all (or, on
+      // failure, release its waits)
+      if (sub == 0) {
+        if (ok && !ensure(nbatch - 1)) fail();
+        for (int b = copied; b < kMaxBatch; ++b) tc_commit(&bsf_ready[b]);
       }
       tc_commit(drain);  // no MMA may still write TMEM when it is freed
       volatile int no_abort = 0;
@@ -395,6 +432,24 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
           for (int j = 0; j < 4; ++j) m = max(m, max((w4[j] << 16) & 0x7FFFFFFFu, w4[j] & 0x7FFF0000u));
         }
       }
+      // The segment is quantized in batches of 256 chunks of 32 elements (one chunk per
+      // thread): chunk c is row (c / 8) % BN, K step c / (8 BN), 32-element piece c % 8,
+      // so that 8 consecutive threads read 512 contiguous bytes of a row and batch b
+      // completes K steps [b kKpb, (b + 1) kKpb).  The first two batches are loaded now:
+      // they arrive while the amax exchange below waits for the other CTAs.
+      const int chunks = BN * seg_steps * 8;
+      auto load_batch = [&](int b, uint4 (&u)[4]) {
+        const int c = b * 256 + xt;
+        const int j = c / (BN * 8), r = (c >> 3) % BN, q = c & 7;
+        const int k = (kb0 + j) * 256 + q * 32;
+        const bool ok = c < chunks && r < p.M && k < p.K;
+        const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.K + k);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) u[e] = ok ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
+      };
+      uint4 ua[4], ub[4];
+      load_batch(0, ua);
+      load_batch(1, ub);
       m = __reduce_max_sync(0xFFFFFFFFu, m);
       if (lane == 0) s_red[xt >> 5] = m;
       named_sync(3, 256);
@@ -460,88 +515,83 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         }
         if (et == 0) *s_abort = 1;
         named_sync(3, 256);
-        if (xt == 0) mbar_arrive(b_ready);
+        if (xt == 0)
+          for (int b = 0; b < kMaxBatch; ++b) mbar_arrive(&b_ready[b]);
       } else {
       const float amax = __uint_as_float(am);
       const float g = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;  // 2688 = 6 * 448
       if (blockIdx.x == 0 && xt == 0 && p.gx_out) *p.gx_out = g;
-      // the segment's codes and scales: one thread per 32 elements (two blocks) of a row
       const bool writer = cta_in_seg == 0;  // writes the segment to the caller's buffers
-      const int chunks = BN * seg_steps * 8;
-      constexpr int CPT = 4;  // chunks per thread in flight at once
-      for (int cb = xt; cb < chunks; cb += 256 * CPT) {
-        uint4 u[CPT][4];
+      // quantize this thread's chunk of batch b: two 16-element blocks of one row
+      auto quantize_batch = [&](int b, const uint4 (&u)[4]) {
+        const int c = b * 256 + xt;
+        if (c >= chunks) return;
+        const int j = c / (BN * 8), r = (c >> 3) % BN, q = c & 7;
+        const int k = (kb0 + j) * 256 + q * 32;
+        uint32_t packed[4];
+        uint32_t sbs[2];
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-          const int c = cb + i * 256;
-          const int r = c / (seg_steps * 8), jc = c % (seg_steps * 8);  // consecutive threads: one row's K
-          const int k = (kb0 + (jc >> 3)) * 256 + (jc & 7) * 32;
-          const bool ok = c < chunks && r < p.M && k < p.K;
-          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.K + k);
+        for (int h = 0; h < 2; ++h) {
+          float v[16];
+          uint32_t bm = 0;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) u[i][e] = ok ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
-        }
+          for (int t = 0; t < 2; ++t) {
+            const uint4 w = u[2 * h + t];
+            const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-          const int c = cb + i * 256;
-          if (c >= chunks) break;
-          const int r = c / (seg_steps * 8);   // row (activation)
-          const int jc = c % (seg_steps * 8);  // 32-element chunk within the row's segment
-          const int j = jc >> 3, q = jc & 7;   // K step within the segment, chunk within it
-          const int k = (kb0 + j) * 256 + q * 32;
-          uint32_t packed[4];
-          uint32_t sbs[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float v[16];
-            uint32_t bm = 0;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const uint4 w = u[i][2 * h + t];
-              const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[t * 8 + 2 * e] = __uint_as_float(w4[e] << 16);
-                v[t * 8 + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
-                bm = max(bm, max((w4[e] << 16) & 0x7FFFFFFFu, w4[e] & 0x7FFF0000u));
-              }
-            }
-            uint32_t sb;
-            const float mul = nvfp4_block_scale(__uint_as_float(bm), g, sb);
-            sbs[h] = sb;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              float sv[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float xe = v[t * 8 + e];
-                sv[e] = xe == 0.0f ? xe : __fmul_rn(xe, mul);  // a zero stays zero if 1/denom overflowed
-              }
-              packed[2 * h + t] = pack8<kE2M1Hardware>(sv);
+            for (int e = 0; e < 4; ++e) {
+              v[t * 8 + 2 * e] = __uint_as_float(w4[e] << 16);
+              v[t * 8 + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+              bm = max(bm, max((w4[e] << 16) & 0x7FFFFFFFu, w4[e] & 0x7FFF0000u));
             }
           }
-          // the operand box of K step j, 128-byte swizzled: 16-byte chunk q of row r
-          *reinterpret_cast<uint4*>(s_b + j * C::kBBox + r * 128 + ((q ^ (r & 7)) << 4)) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          // scale bytes: blocks 2q and 2q+1 of the K step -> atom (j, q / 2), column 2 (q % 2) + h
+          uint32_t sb;
+          const float mul = nvfp4_block_scale(__uint_as_float(bm), g, sb);
+          sbs[h] = sb;
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            s_bsf[(j * 4 + (q >> 1)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + ((q & 1) * 2 + h)] =
-                static_cast<uint8_t>(sbs[h]);
-          if (writer && r < p.M && k < p.K)
-            *reinterpret_cast<uint4*>(p.xq_out + static_cast<int64_t>(r) * (p.K / 2) + k / 2) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          for (int t = 0; t < 2; ++t) {
+            float sv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float xe = v[t * 8 + e];
+              sv[e] = xe == 0.0f ? xe : __fmul_rn(xe, mul);  // a zero stays zero if 1/denom overflowed
+            }
+            packed[2 * h + t] = pack8<kE2M1Hardware>(sv);
+          }
+        }
+        // the operand box of K step j, 128-byte swizzled: 16-byte chunk q of row r
+        *reinterpret_cast<uint4*>(s_b + j * C::kBBox + r * 128 + ((q ^ (r & 7)) << 4)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        // scale bytes: blocks 2q and 2q+1 of the K step -> atom (j, q / 2), column 2 (q % 2) + h
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          s_bsf[(j * 4 + (q >> 1)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + ((q & 1) * 2 + h)] =
+              static_cast<uint8_t>(sbs[h]);
+        if (writer && r < p.M && k < p.K)
+          *reinterpret_cast<uint4*>(p.xq_out + static_cast<int64_t>(r) * (p.K / 2) + k / 2) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      };
+      // batch b is in shared memory: make it visible to the tensor cores and announce it
+      auto publish = [&](int b) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
+        named_sync(3, 256);
+        if (xt == 0) mbar_arrive(&b_ready[b]);
+      };
+      for (int b = 0; b < nbatch; b += 2) {
+        quantize_batch(b, ua);
+        publish(b);
+        if (b + 2 < nbatch) load_batch(b + 2, ua);
+        if (b + 1 < nbatch) {
+          quantize_batch(b + 1, ub);
+          publish(b + 1);
+          if (b + 3 < nbatch) load_batch(b + 3, ub);
         }
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
-      named_sync(3, 256);
       if (writer) {  // the segment's scale atoms (pads included) to the caller's buffer
-        const int atoms = min(seg_steps * 4, p.atoms_k - kb0 * 4);
-        for (int o = xt; o < atoms * 32; o += 256)
+        for (int o = xt; o < seg_atoms * 32; o += 256)
           reinterpret_cast<uint4*>(p.xs_out + static_cast<int64_t>(kb0) * 4 * 512)[o] =
               reinterpret_cast<const uint4*>(s_bsf)[o];
       }
-      if (xt == 0) mbar_arrive(b_ready);
       }
     }
     // ------------------------------------------------------------ epilogue

@@ -563,11 +563,18 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       const int row = w.out_row0 + rl;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
       if (q * 32 < w.rows_valid) {  // warp-uniform: warps without a valid row skip TMEM
+        // up to 64 columns per TMEM round trip: four loads in flight, one wait
+        constexpr int CW = BN >= 64 ? 64 : BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(taddr + c, r);
+        for (int cw = 0; cw < BN; cw += CW) {
+          uint32_t rr[CW / 16][16];
+#pragma unroll
+          for (int h = 0; h < CW / 16; ++h) tmem_ld16(taddr + cw + h * 16, rr[h]);
           tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < CW / 16; ++h) {
+          const int c = cw + h * 16;
+          const uint32_t (&r)[16] = rr[h];
           const int col = w.n0 + c;
           if (!row_ok || col >= p.Nk) continue;
           if (p.mode == kModeStreamK) {
@@ -586,6 +593,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]) * scale;
             store_row16(p, row, col, v);
           }
+        }
         }
       }
       tc_fence_before();
@@ -754,15 +762,19 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
     pl.swap = false;
     pl.Mk = M;
     pl.Nk = N;
-    pl.BN = N >= 256 ? 256 : 128;
+    // 256-wide tiles when there are enough of them to fill the SMs, else 128-wide
+    const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
+    pl.BN = (N >= 256 && tiles256 >= num_sms()) ? 256 : 128;
     pl.ACC = pl.BN == 256 ? 1 : 2;
   }
   pl.tiles_m = static_cast<int>((pl.Mk + 127) / 128);
   pl.tiles_n = static_cast<int>((pl.Nk + pl.BN - 1) / pl.BN);
   const int64_t tiles = static_cast<int64_t>(pl.tiles_m) * pl.tiles_n;
   const int sms = num_sms();
-  // too few tiles to fill the SMs: split every tile's K range across CTAs (stream-K)
-  if (tiles < 2 * sms && pl.num_kb >= 4) {
+  // Too few tiles to fill the SMs: split every tile's K range across CTAs (stream-K).
+  // Swapped (decode-like) shapes split whenever tiles are scarce; the others only when
+  // K is long enough that the split's partial-sum traffic stays small against the MMAs.
+  if (tiles < 2 * sms && pl.num_kb >= 4 && (pl.swap || (2 * tiles < sms && pl.num_kb >= 16))) {
     pl.mode = kModeStreamK;
     pl.units = tiles * pl.num_kb;
     pl.ws_bytes = (static_cast<size_t>(M * N) * 4 + 255) / 256 * 256 + (static_cast<size_t>(tiles) * 4 + 255) / 256 * 256;

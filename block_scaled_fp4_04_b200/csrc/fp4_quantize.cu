@@ -492,19 +492,28 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
   constexpr int CPR = 128 / EPC;
   unsigned bad = 0;
 
-  // stage the region
-  for (int idx = tid; idx < 128 * CPR; idx += 256) {
-    const int rl = idx / CPR, ch = idx % CPR;
-    const int64_t r = r0 + rl, c = c0 + ch * EPC;
-    float v[EPC];
-    if (r < p.rows && c < p.cols) {
-      Elem<T>::unpack(ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + c) * sizeof(T)), v);
-    } else {
+  // stage the region, eight 16-byte loads in flight per thread
+  constexpr int NLD = 8;
+  static_assert((128 * CPR) % (256 * NLD) == 0, "staging loop");
+  for (int base = tid; base < 128 * CPR; base += 256 * NLD) {
+    uint4 u[NLD];
 #pragma unroll
-      for (int i = 0; i < EPC; ++i) v[i] = 0.0f;
+    for (int j = 0; j < NLD; ++j) {
+      const int idx = base + j * 256;
+      const int rl = idx / CPR, ch = idx % CPR;
+      const int64_t r = r0 + rl, c = c0 + ch * EPC;
+      u[j] = (r < p.rows && c < p.cols) ? ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + c) * sizeof(T))
+                                        : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int i = 0; i < EPC; ++i) s_x[rl * LD + ch * EPC + i] = v[i];
+    for (int j = 0; j < NLD; ++j) {
+      const int idx = base + j * 256;
+      const int rl = idx / CPR, ch = idx % CPR;
+      float v[EPC];
+      Elem<T>::unpack(u[j], v);
+#pragma unroll
+      for (int i = 0; i < EPC; ++i) s_x[rl * LD + ch * EPC + i] = v[i];
+    }
   }
   __syncthreads();
   // patch amax: 4 threads per patch, 4 rows each

@@ -107,6 +107,8 @@ GEMM_CASES = [
     (40, 640, 2048, fp4.NVFP4, torch.float32),       # swapped with N-tile 64
     (64, 384, 8192, fp4.MXFP4, torch.bfloat16),
     (1024, 1024, 1024, fp4.NVFP4, torch.bfloat16),   # training sweep, smallest square
+    (256, 256, 8192, fp4.NVFP4, torch.float32),      # few tiles, long K: split over K
+    (130, 384, 4096, fp4.NVFP4, torch.bfloat16),     # split over K with a ragged M tile
 ]
 
 
