@@ -625,6 +625,72 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
       named_sync(1 + sub, 128);  // the list is reused
       npend = 0;
     };
+    // Write-out.  Tile t belongs to pipeline t mod (pipelines in the grid).  Its owner
+    // waits (bounded) until the tile's counter shows every K step summed, then scales,
+    // converts and stores the tile and clears the sums and the counter behind it.  (The
+    // launch is cooperative, so an owner never waits for a CTA that cannot run.)
+    const int gp = blockIdx.x * C::kP + sub, np = gridDim.x * C::kP;
+    int next_owned = gp;
+    auto write_owned = [&]() {
+      while (next_owned < p.tiles && !*s_epi_fail && !*s_xfail) {
+        const int t = next_owned;
+        if (et == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          int ready = 0;
+          for (uint32_t it = 1; it < kWaitMaxIters; ++it) {
+            int c;
+            asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(c) : "l"(p.tile_cnt + t) : "memory");
+            if (c >= p.num_kb) {
+              ready = 1;
+              break;
+            }
+            if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+              d_latch_timeout(s_abort, p.status);
+              *s_epi_fail = 1;
+              break;
+            }
+            __nanosleep(64);
+          }
+          if (ready) __threadfence();
+          *s_last = ready;
+        }
+        named_sync(1 + sub, 128);
+        const int ready = *s_last;
+        named_sync(1 + sub, 128);  // s_last is rewritten on the next turn
+        if (*s_epi_fail || !ready) return;
+        const int row = t * 128 + rl;
+        if (row < p.N) {
+          float* wsrow = p.ws + static_cast<int64_t>(row) * p.M;
+          float v[BN];
+          if ((p.M & 3) == 0) {
+#pragma unroll
+            for (int j = 0; j < BN; j += 4)
+              if (j < p.M) {
+                const float4 f = __ldcg(reinterpret_cast<const float4*>(wsrow + j));
+                v[j] = f.x;
+                v[j + 1] = f.y;
+                v[j + 2] = f.z;
+                v[j + 3] = f.w;
+              }
+#pragma unroll
+            for (int j = 0; j < BN; j += 4)
+              if (j < p.M) __stcg(reinterpret_cast<float4*>(wsrow + j), make_float4(0.f, 0.f, 0.f, 0.f));
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN; ++j)
+              if (j < p.M) v[j] = __ldcg(wsrow + j);
+#pragma unroll
+            for (int j = 0; j < BN; ++j)
+              if (j < p.M) __stcg(wsrow + j, 0.0f);
+          }
+#pragma unroll
+          for (int j = 0; j < BN; ++j)
+            if (j < p.M) d_store(p, row, j, v[j] * scale);
+        }
+        if (et == 0) p.tile_cnt[t] = 0;
+        next_owned += np;
+      }
+    };
     DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg);
     int tile, k0, k1, iter = 0;
     while (!*s_xfail && sch.next(tile, k0, k1)) {
@@ -668,64 +734,7 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
       if (++npend == kMaxPend) flush();
     }
     if (npend && !*s_epi_fail && !*s_xfail) flush();
-    // Write-out.  Tile t belongs to pipeline t mod (pipelines in the grid); its owner waits
-    // until the tile's counter shows every K step summed, then scales, converts and
-    // stores it and clears the sums and the counter behind it.  (All CTAs are resident:
-    // the launch is cooperative, so an owner never waits for a CTA that cannot run.)
-    const int gp = blockIdx.x * C::kP + sub, np = gridDim.x * C::kP;
-    for (int t = gp; t < p.tiles && !*s_epi_fail && !*s_xfail; t += np) {
-      if (et == 0) {
-        const uint64_t t0 = globaltimer_ns();
-        bool done = false;
-        for (uint32_t it = 1; it < kWaitMaxIters; ++it) {
-          int c;
-          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(c) : "l"(p.tile_cnt + t) : "memory");
-          if (c >= p.num_kb) {
-            done = true;
-            break;
-          }
-          if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) break;
-          __nanosleep(64);
-        }
-        if (!done) {
-          d_latch_timeout(s_abort, p.status);
-          *s_epi_fail = 1;
-        }
-        __threadfence();
-      }
-      named_sync(1 + sub, 128);
-      if (*s_epi_fail) break;
-      const int row = t * 128 + rl;
-      if (row < p.N) {
-        float* wsrow = p.ws + static_cast<int64_t>(row) * p.M;
-        float v[BN];
-        if ((p.M & 3) == 0) {
-#pragma unroll
-          for (int j = 0; j < BN; j += 4)
-            if (j < p.M) {
-              const float4 f = __ldcg(reinterpret_cast<const float4*>(wsrow + j));
-              v[j] = f.x;
-              v[j + 1] = f.y;
-              v[j + 2] = f.z;
-              v[j + 3] = f.w;
-            }
-#pragma unroll
-          for (int j = 0; j < BN; j += 4)
-            if (j < p.M) __stcg(reinterpret_cast<float4*>(wsrow + j), make_float4(0.f, 0.f, 0.f, 0.f));
-        } else {
-#pragma unroll
-          for (int j = 0; j < BN; ++j)
-            if (j < p.M) v[j] = __ldcg(wsrow + j);
-#pragma unroll
-          for (int j = 0; j < BN; ++j)
-            if (j < p.M) __stcg(wsrow + j, 0.0f);
-        }
-#pragma unroll
-        for (int j = 0; j < BN; ++j)
-          if (j < p.M) d_store(p, row, j, v[j] * scale);
-      }
-      if (et == 0) p.tile_cnt[t] = 0;
-    }
+    write_owned();
   }
 
   tc_fence_before();

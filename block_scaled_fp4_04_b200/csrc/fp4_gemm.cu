@@ -742,13 +742,16 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
   pl.num_kb = static_cast<int>((K + 255) / 256);
   (void)mx;
   if (grouped) {
+    // 256-wide tiles: per MMA the scale-factor copies into TMEM cost less than with
+    // 128-wide ones (an expert's last N-tile may be half empty; its extra columns, read
+    // from the next expert's rows, are never stored)
     pl.swap = false;
-    pl.BN = 128;
-    pl.ACC = 2;
+    pl.BN = N >= 256 ? 256 : 128;
+    pl.ACC = pl.BN == 256 ? 1 : 2;
     pl.mode = kModeGrouped;
     pl.Mk = M;
     pl.Nk = N;
-    pl.tiles_n = static_cast<int>(N / 128);
+    pl.tiles_n = static_cast<int>((N + pl.BN - 1) / pl.BN);
     pl.ws_bytes = 0;
     return pl;
   }
