@@ -108,6 +108,9 @@ GEMM_CASES = [
     (64, 384, 8192, fp4.MXFP4, torch.bfloat16),
     (1024, 1024, 1024, fp4.NVFP4, torch.bfloat16),   # training sweep, smallest square
     (256, 256, 8192, fp4.NVFP4, torch.float32),      # few tiles, long K: split over K
+    (16, 1000, 2048, fp4.NVFP4, torch.bfloat16),     # decode kernel, ragged last weight tile
+    (32, 200, 8192, fp4.NVFP4, torch.float32),       # decode kernel, N-tile 32, few tiles
+    (7, 640, 2080, fp4.NVFP4, torch.bfloat16),       # decode kernel, K tail (2080 = 8*256 + 32)
     (130, 384, 4096, fp4.NVFP4, torch.bfloat16),     # split over K with a ragged M tile
 ]
 
@@ -253,7 +256,8 @@ def _bf16a(xa, qb, n, k, out_dtype=torch.bfloat16, flags=0, ws=None):
 
 
 @pytest.mark.parametrize("m,n,k,flags", [(16, 1024, 4096, 0), (16, 1024, 4096, 1), (1, 256, 256, 0),
-                                         (32, 512, 2048, 1), (5, 384, 96, 0), (200, 256, 512, 1)])
+                                         (32, 512, 2048, 1), (5, 384, 96, 0), (200, 256, 512, 1),
+                                         (20, 1000, 2080, 1), (16, 384, 16384, 0)])
 def test_gemm_bf16a_matches_oracle(m, n, k, flags):
     """Activations quantized inside the call: codes, scales and g bit-exact; D in tolerance."""
     from fp4_testutil import assert_quant_equal
