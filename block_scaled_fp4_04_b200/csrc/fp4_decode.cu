@@ -56,11 +56,16 @@ struct DecodeArgs {
   unsigned* status;
 };
 
+// K steps of one segment at most (the activations' scale factors for a segment take 16
+// TMEM columns per K step; longer segments measured slower: fewer partial sums, but each
+// CTA quantizes twice as much of X and its rings are shallower)
+constexpr int decode_max_seg(int) { return 8; }
+
 template <int BN>
 struct DecodeCfg {
   static constexpr int kP = 2;                              // pipelines per CTA
   static constexpr int kThreads = 192 * kP;
-  static constexpr int kMaxSeg = 8;                         // K steps of one segment (max)
+  static constexpr int kMaxSeg = decode_max_seg(BN);        // K steps of one segment (max)
   static constexpr int kBBox = BN * 128;                    // one K step of activation codes
   static constexpr int kBBytes = kMaxSeg * kBBox;
   static constexpr int kBSFBytes = kMaxSeg * 4 * 512;
@@ -114,19 +119,35 @@ __device__ __forceinline__ void d_store(const DecodeArgs& p, int row, int col, f
 
 // The (weight tile, K step) units of one pipeline: units u in [u0, u1) of its segment,
 // u -> tile u / seg_len, K step kb0 + u % seg_len; consecutive units of one tile form
-// one accumulation.
+// one accumulation.  In the fused kernel a range that starts inside a tile (and goes on
+// past it) takes that partial tile last, so that the pipeline starts on the segment's
+// first K step -- the one whose activations are quantized first.  (With pre-quantized
+// activations every K step is ready at once and the natural order finishes tiles sooner.)
 struct DecodeSched {
   int64_t u, u1;
+  int64_t head0, head1;  // the deferred partial first tile: units [head0, head1), or empty
   int kb0, len;
-  __device__ DecodeSched(const DecodeArgs& p, int seg, int pipe_in_seg, int pipes_in_seg) {
+  __device__ DecodeSched(const DecodeArgs& p, int seg, int pipe_in_seg, int pipes_in_seg, bool defer_head) {
     kb0 = seg * p.seg_len;
     len = min(p.seg_len, p.num_kb - kb0);
     const int64_t U = static_cast<int64_t>(p.tiles) * len;
     u = U * pipe_in_seg / pipes_in_seg;
     u1 = U * (pipe_in_seg + 1) / pipes_in_seg;
+    head0 = head1 = 0;
+    const int64_t first_end = (u / len + 1) * len;
+    if (defer_head && u % len != 0 && u1 > first_end) {
+      head0 = u;
+      head1 = first_end;
+      u = first_end;
+    }
   }
   // next accumulation: tile, K steps [k0, k1)
   __device__ bool next(int& tile, int& k0, int& k1) {
+    if (u >= u1 && head0 < head1) {
+      u = head0;
+      u1 = head1;
+      head0 = head1 = 0;
+    }
     if (u >= u1) return false;
     tile = static_cast<int>(u / len);
     const int j0 = static_cast<int>(u % len);
@@ -245,7 +266,7 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         d_wait_prior_grids();
         load_x();
       }
-      DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg);
+      DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg, FUSED);
       int tile, k0, k1, stage = 0, issued_n = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
       bool ok = true, x_done = !p.weights_ready;
@@ -327,10 +348,6 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
             if (!mbar_wait(&b_ready[copied], 0, s_abort) || *s_xfail) return false;
             copy_batch(copied++);
           }
-          while (copied < nbatch && mbar_try_wait(&b_ready[copied], 0)) {
-            if (*s_xfail) return false;
-            copy_batch(copied++);
-          }
           return true;  // this thread's own copies precede its MMAs
         }
         while (known <= need) {
@@ -340,12 +357,18 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         tc_fence_after();
         return true;
       };
+      // later batches that are already quantized: copied after a stage's MMAs are issued,
+      // so that they never delay an MMA that does not need them
+      auto copy_ready = [&]() {
+        if (sub != 0) return;
+        while (copied < nbatch && !*s_xfail && mbar_try_wait(&b_ready[copied], 0)) copy_batch(copied++);
+      };
       auto fail = [&]() {
         if (!*s_xfail) d_latch_timeout(s_abort, p.status);
         ok = false;
       };
       if (!ensure(0)) fail();
-      DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg);
+      DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg, FUSED);
       const uint32_t ring_s = smem_u32(ring), b_s = smem_u32(s_b);
       int tile, k0, k1, stage = 0, iter = 0;
       uint32_t phase = 0, slot = 0;
@@ -382,6 +405,7 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
             tc_mma_nvfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t + k * 4, sfb_t + k * 4,
                          (kb > k0 || k > 0) ? 1u : 0u);
           tc_commit(&empty[stage]);
+          copy_ready();
           slot ^= 1;
           if (++stage == S) {
             stage = 0;
@@ -691,7 +715,7 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         next_owned += np;
       }
     };
-    DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg);
+    DecodeSched sch(p, seg, pipe_in_seg, pipes_in_seg, FUSED);
     int tile, k0, k1, iter = 0;
     while (!*s_xfail && sch.next(tile, k0, k1)) {
       const int acc = iter % C::kACC;
@@ -754,14 +778,16 @@ struct DecodePlan {
   int nseg, seg_len, ctas_per_seg, tiles, num_kb;
 };
 
-static DecodePlan decode_plan(int64_t N, int64_t K) {
+static DecodePlan decode_plan(int64_t N, int64_t K, int bn) {
   DecodePlan d{};
   d.num_kb = static_cast<int>((K + 255) / 256);
   d.tiles = static_cast<int>((N + 127) / 128);
   const int sms = num_sms();
-  // segments of at most 8 K steps; enough segments that every SM gets a CTA
-  int nseg = (d.num_kb + 7) / 8;
-  if (nseg < 4) nseg = d.num_kb < 4 ? d.num_kb : 4;
+  // segments of at most decode_max_seg(bn) K steps
+  const int max_seg = decode_max_seg(bn);
+  int nseg = (d.num_kb + max_seg - 1) / max_seg;
+  const int min_seg = 4;
+  if (nseg < min_seg) nseg = d.num_kb < min_seg ? d.num_kb : min_seg;
   if (nseg > sms) nseg = sms;
   const int max_ctas = sms < kDecodeMaxCtas ? sms : kDecodeMaxCtas;
   d.seg_len = (d.num_kb + nseg - 1) / nseg;
@@ -822,8 +848,8 @@ int launch_decode(const DecodeProblem& q, unsigned* status, cudaStream_t st, con
     *why = "workspace too small (see fp4_gemm_workspace_size)";
     return 1;
   }
-  const DecodePlan pl = decode_plan(q.N, q.K);
   const int BN = q.M <= 16 ? 16 : 32;
+  const DecodePlan pl = decode_plan(q.N, q.K, BN);
   CUtensorMap tw, tx;
   if (!make_tensor_map_u8(&tw, q.W, static_cast<uint64_t>(q.K / 2), static_cast<uint64_t>(q.N), 128)) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
