@@ -196,7 +196,11 @@ constexpr int pipes_per_cta() { return BN <= 32 ? FP4_SMALL_N_PIPES : BN <= 64 ?
 template <int BN, bool MX, int ACC>
 struct Cfg {
   static constexpr int kP = pipes_per_cta<BN>();
-  static constexpr int kThreads = 192 * kP;
+  // Single-pipeline kernels (128/256-wide tiles) add a seventh warp that copies each
+  // stage's scale factors into TMEM, so that these copies are not serialised behind the
+  // MMA thread's own MMAs.
+  static constexpr bool kSepCp = kP == 1;
+  static constexpr int kThreads = kSepCp ? 224 : 192 * kP;
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
@@ -301,8 +305,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
-  const int sub = threadIdx.x / 192;  // pipeline of this thread
-  const int lt = threadIdx.x % 192;
+  const int sub = C::kP == 1 ? 0 : threadIdx.x / 192;  // pipeline of this thread
+  const int lt = C::kP == 1 ? threadIdx.x : threadIdx.x % 192;
   const int warp = lt >> 5, lane = lt & 31;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023)) +
                   sub * C::kSubBytes;
@@ -312,7 +316,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   uint64_t* acc_full = empty + S;
   uint64_t* acc_empty = acc_full + ACC;
   uint64_t* drain = acc_empty + ACC;
-  volatile int* s_abort = reinterpret_cast<volatile int*>(drain + 1);
+  uint64_t* sf_full = drain + 1;     // [2]: a stage's scale factors are in TMEM slot i
+  uint64_t* cp_drain = sf_full + 2;  // the copier's last copies have completed
+  volatile int* s_abort = reinterpret_cast<volatile int*>(cp_drain + 1);
   volatile int* s_epi_fail = s_abort + 1;
   volatile int* s_last = s_abort + 2;  // stream-K: this pipeline completes the current tile
   int* s_mt = reinterpret_cast<int*>(misc + 1024);
@@ -330,6 +336,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       mbar_init(&acc_empty[a], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(&sf_full[0], 1);
+    mbar_init(&sf_full[1], 1);
+    mbar_init(cp_drain, 1);
     *s_abort = 0;
     *s_epi_fail = 0;
     *s_last = 0;
@@ -377,6 +386,17 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem_base + sub * C::kTmemCols;
   const uint32_t sf_col0 = ACC * BN;
+  // copies one stage's scale-factor atoms (A's, then B's row-blocks) into a TMEM slot
+  auto copy_stage_sf = [&](uint32_t st, uint32_t sfa_t, int kb) {
+    const uint32_t sfb_t = sfa_t + C::kSFACols;
+    const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+    for (int a = 0; a < atoms; ++a) tc_cp_sf_atom(sfa_t + a * 4, smem_desc_sf(st + C::kABytes + C::kBBytes + a * 512));
+#pragma unroll
+    for (int rb = 0; rb < C::kNRB; ++rb)
+      for (int a = 0; a < atoms; ++a)
+        tc_cp_sf_atom(sfb_t + (a * C::kNRB + rb) * 4,
+                      smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -473,7 +493,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       Sched<BN> sch(p, s_mt, s_off, vb, vg);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
-      int stage = 0, iter = 0;
+      int stage = 0, iter = 0, nstage = 0;
       uint32_t phase = 0, slot = 0;
       bool ok = true;
       while (ok && sch.next(w)) {
@@ -490,18 +510,22 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint32_t st = smem_base + stage * C::kStageBytes;
           const uint32_t sfa_t = tmem + sf_col0 + slot * C::kSFSlot;
           const uint32_t sfb_t = sfa_t + C::kSFACols;
-          const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
-          for (int a = 0; a < atoms; ++a)
-            tc_cp_sf_atom(sfa_t + a * 4, smem_desc_sf(st + C::kABytes + C::kBBytes + a * 512));
-#pragma unroll
-          for (int rb = 0; rb < C::kNRB; ++rb)
-            for (int a = 0; a < atoms; ++a)
-              tc_cp_sf_atom(sfb_t + (a * C::kNRB + rb) * 4,
-                            smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
+          if constexpr (C::kSepCp) {
+            // the copier has put this stage's scale factors into the slot
+            if (!mbar_wait(&sf_full[slot], (nstage >> 1) & 1, s_abort)) {
+              latch_timeout(s_abort, p.status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          } else {
+            tc_fence_after();
+            copy_stage_sf(st, sfa_t, kb);
+          }
+          ++nstage;
           const int krem = p.K - kb * 256;
           const int nk = krem >= 256 ? 4 : (krem + 63) / 64;
           const uint64_t adesc = smem_desc_sw128(st);
@@ -534,7 +558,50 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
-  } else {
+  } else if (C::kSepCp && warp == 6) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ scale-factor copier
+      // Stage n's atoms go to TMEM slot n % 2 once the stage has landed and the MMAs of
+      // stage n - 2 (the slot's previous user) have completed; each slot's copies are
+      // committed to sf_full[slot] for the MMA thread.
+      Sched<BN> sch(p, s_mt, s_off, vb, vg);
+      const uint32_t smem_base = smem_u32(smem);
+      Work w;
+      int stage = 0, n = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      while (ok && sch.next(w)) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort)) {
+            latch_timeout(s_abort, p.status);
+            ok = false;
+            break;
+          }
+          if (n >= 2) {
+            const int prev = n - 2;
+            if (!mbar_wait(&empty[prev % S], (prev / S) & 1, s_abort)) {
+              latch_timeout(s_abort, p.status);
+              ok = false;
+              break;
+            }
+          }
+          tc_fence_after();
+          const uint32_t sl = n & 1;
+          copy_stage_sf(smem_base + stage * C::kStageBytes, tmem + sf_col0 + sl * C::kSFSlot, kb);
+          tc_commit(&sf_full[sl]);
+          ++n;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // no copy may still write TMEM when it is freed
+      tc_commit(cp_drain);
+      volatile int no_abort = 0;
+      mbar_wait(cp_drain, 0, &no_abort);
+    }
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     // a warp reads the TMEM lane quarter given by its warp index in the CTA, modulo 4
     const int q = (threadIdx.x >> 5) & 3;
