@@ -222,13 +222,19 @@ struct Cfg {
   static constexpr int kSFACols = kAtomsKT * 4;
   static constexpr int kSFBCols = kNRB * kAtomsKT * 4;
   static constexpr int kSFSlot = kSFACols + kSFBCols;
-  static constexpr int kColsUsed = ACC * BN + 2 * kSFSlot;
+  // TMEM slots for the stages' scale factors: with a separate copier, as many as fit
+  // (up to 4, and fewer than the ring's stages) so that it can run ahead of the MMAs
+  static constexpr int kSlotsFit = (512 - ACC * BN) / kSFSlot;
+  static constexpr int kSFSlots = !kSepCp ? 2 : (kSlotsFit < 4 ? kSlotsFit : 4) < kStages ? (kSlotsFit < 4 ? kSlotsFit : 4)
+                                                                                           : kStages - 1;
+  static constexpr int kColsUsed = ACC * BN + kSFSlots * kSFSlot;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;  // per pipeline
   // one allocation for all pipelines: a power of two of at least 32 columns
   static constexpr int kTmemAlloc = kP * kTmemCols <= 32 ? 32 : kP * kTmemCols <= 64 ? 64
                                     : kP * kTmemCols <= 128 ? 128 : kP * kTmemCols <= 256 ? 256 : 512;
   static_assert(kP * kTmemCols <= 512, "TMEM budget");
+  static_assert(kSFSlots >= 2 && kSFSlots < kStages, "scale-factor slots");
   static_assert(kStageBytes % 1024 == 0 && kSubBytes % 1024 == 0, "128-byte swizzled stages need 1024-byte alignment");
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -316,8 +322,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   uint64_t* acc_full = empty + S;
   uint64_t* acc_empty = acc_full + ACC;
   uint64_t* drain = acc_empty + ACC;
-  uint64_t* sf_full = drain + 1;     // [2]: a stage's scale factors are in TMEM slot i
-  uint64_t* cp_drain = sf_full + 2;  // the copier's last copies have completed
+  uint64_t* sf_full = drain + 1;                // [kSFSlots]: stage scale factors are in TMEM slot i
+  uint64_t* cp_drain = sf_full + C::kSFSlots;   // the copier's last copies have completed
   volatile int* s_abort = reinterpret_cast<volatile int*>(cp_drain + 1);
   volatile int* s_epi_fail = s_abort + 1;
   volatile int* s_last = s_abort + 2;  // stream-K: this pipeline completes the current tile
@@ -336,8 +342,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       mbar_init(&acc_empty[a], 4);
     }
     mbar_init(drain, 1);
-    mbar_init(&sf_full[0], 1);
-    mbar_init(&sf_full[1], 1);
+    for (int i = 0; i < C::kSFSlots; ++i) mbar_init(&sf_full[i], 1);
     mbar_init(cp_drain, 1);
     *s_abort = 0;
     *s_epi_fail = 0;
@@ -515,7 +520,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
           const uint32_t sfb_t = sfa_t + C::kSFACols;
           if constexpr (C::kSepCp) {
             // the copier has put this stage's scale factors into the slot
-            if (!mbar_wait(&sf_full[slot], (nstage >> 1) & 1, s_abort)) {
+            if (!mbar_wait(&sf_full[slot], (nstage / C::kSFSlots) & 1, s_abort)) {
               latch_timeout(s_abort, p.status);
               ok = false;
               break;
@@ -543,7 +548,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
               tc_mma_nvfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
           }
           tc_commit(&empty[stage]);
-          slot ^= 1;
+          if (++slot == C::kSFSlots) slot = 0;
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
@@ -561,9 +566,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   } else if (C::kSepCp && warp == 6) {
     if (lane == 0) {
       // ------------------------------------------------------------ scale-factor copier
-      // Stage n's atoms go to TMEM slot n % 2 once the stage has landed and the MMAs of
-      // stage n - 2 (the slot's previous user) have completed; each slot's copies are
-      // committed to sf_full[slot] for the MMA thread.
+      // Stage n's atoms go to TMEM slot n % kSFSlots once the stage has landed and the
+      // MMAs of stage n - kSFSlots (the slot's previous user) have completed; each slot's
+      // copies are committed to sf_full[slot] for the MMA thread.
       Sched<BN> sch(p, s_mt, s_off, vb, vg);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
@@ -577,8 +582,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             ok = false;
             break;
           }
-          if (n >= 2) {
-            const int prev = n - 2;
+          if (n >= C::kSFSlots) {
+            const int prev = n - C::kSFSlots;
             if (!mbar_wait(&empty[prev % S], (prev / S) & 1, s_abort)) {
               latch_timeout(s_abort, p.status);
               ok = false;
@@ -586,7 +591,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             }
           }
           tc_fence_after();
-          const uint32_t sl = n & 1;
+          const uint32_t sl = n % C::kSFSlots;
           copy_stage_sf(smem_base + stage * C::kStageBytes, tmem + sf_col0 + sl * C::kSFSlot, kb);
           tc_commit(&sf_full[sl]);
           ++n;
