@@ -196,11 +196,12 @@ constexpr int pipes_per_cta() { return BN <= 32 ? FP4_SMALL_N_PIPES : BN <= 64 ?
 template <int BN, bool MX, int ACC>
 struct Cfg {
   static constexpr int kP = pipes_per_cta<BN>();
-  // Single-pipeline kernels (128/256-wide tiles) add a seventh warp that copies each
-  // stage's scale factors into TMEM, so that these copies are not serialised behind the
-  // MMA thread's own MMAs.
+  // Single-pipeline kernels (128/256-wide tiles) add copier warps that move each stage's
+  // scale factors into TMEM, so that these copies are not serialised behind the MMA
+  // thread's own MMAs: one for A's atoms and one per 128-row block of B's.
   static constexpr bool kSepCp = kP == 1;
-  static constexpr int kThreads = kSepCp ? 224 : 192 * kP;
+  static constexpr int kCopiers = kSepCp ? 1 + (BN >= 128 ? BN / 128 : 1) : 0;
+  static constexpr int kThreads = kSepCp ? 192 + 32 * kCopiers : 192 * kP;
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
@@ -342,8 +343,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       mbar_init(&acc_empty[a], 4);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < C::kSFSlots; ++i) mbar_init(&sf_full[i], 1);
-    mbar_init(cp_drain, 1);
+    for (int i = 0; i < C::kSFSlots; ++i) mbar_init(&sf_full[i], C::kSepCp ? C::kCopiers : 1);
+    mbar_init(cp_drain, C::kSepCp ? C::kCopiers : 1);
     *s_abort = 0;
     *s_epi_fail = 0;
     *s_last = 0;
@@ -563,7 +564,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
-  } else if (C::kSepCp && warp == 6) {
+  } else if (C::kSepCp && warp >= 6) {
+    const int cw = warp - 6;  // 0: A's atoms; 1 + rb: B's row-block rb
     if (lane == 0) {
       // ------------------------------------------------------------ scale-factor copier
       // Stage n's atoms go to TMEM slot n % kSFSlots once the stage has landed and the
@@ -592,7 +594,20 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sl = n % C::kSFSlots;
-          copy_stage_sf(smem_base + stage * C::kStageBytes, tmem + sf_col0 + sl * C::kSFSlot, kb);
+          {
+            const uint32_t st = smem_base + stage * C::kStageBytes;
+            const uint32_t sfa_t = tmem + sf_col0 + sl * C::kSFSlot;
+            const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+            if (cw == 0) {
+              for (int a = 0; a < atoms; ++a)
+                tc_cp_sf_atom(sfa_t + a * 4, smem_desc_sf(st + C::kABytes + C::kBBytes + a * 512));
+            } else {
+              const int rb = cw - 1;
+              for (int a = 0; a < atoms; ++a)
+                tc_cp_sf_atom(sfa_t + C::kSFACols + (a * C::kNRB + rb) * 4,
+                              smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
+            }
+          }
           tc_commit(&sf_full[sl]);
           ++n;
           if (++stage == S) {
