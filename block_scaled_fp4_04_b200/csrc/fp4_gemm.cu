@@ -201,7 +201,12 @@ struct Cfg {
   // thread's own MMAs: one for A's atoms and one per 128-row block of B's.
   static constexpr bool kSepCp = kP == 1;
   static constexpr int kCopiers = kSepCp ? 1 + (BN >= 128 ? BN / 128 : 1) : 0;
-  static constexpr int kThreads = kSepCp ? 192 + 32 * kCopiers : 192 * kP;
+  // One-pipeline kernels run two epilogue warps per TMEM lane quarter, one per column
+  // half: twice the TMEM read and store rate, and half a row of packed BF16 per thread
+  // is few enough registers to hold the tile while TMEM is already handed back.
+  static constexpr int kEpiWarps = kSepCp ? 8 : 4;
+  static constexpr int kEpiCols = BN * 4 / kEpiWarps;  // accumulator columns per epilogue thread
+  static constexpr int kThreads = kSepCp ? 64 + 32 * kEpiWarps + 32 * kCopiers : 192 * kP;
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
@@ -299,9 +304,9 @@ __device__ __forceinline__ void store_row16(const GemmArgs& p, int row, int col,
     if (col + j < p.Nk) store_out(p, base + j, v[j]);
 }
 
-// Named barrier among the 128 epilogue threads of one pipeline.
-__device__ __forceinline__ void epi_sync(int sub) {
-  asm volatile("bar.sync %0, 128;" ::"r"(1 + sub) : "memory");
+// Named barrier among the epilogue threads of one pipeline.
+__device__ __forceinline__ void epi_sync(int sub, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + sub), "r"(nthreads) : "memory");
 }
 
 template <int BN, bool MX, int ACC>
@@ -325,7 +330,11 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   uint64_t* drain = acc_empty + ACC;
   uint64_t* sf_full = drain + 1;                // [kSFSlots]: stage scale factors are in TMEM slot i
   uint64_t* cp_drain = sf_full + C::kSFSlots;   // the copier's last copies have completed
-  volatile int* s_abort = reinterpret_cast<volatile int*>(cp_drain + 1);
+  // [S]: a stage's scale factors have landed.  With a separate copier they complete on
+  // their own barrier (and are issued first), so that the copier moves them into TMEM
+  // while the stage's operand tiles are still arriving; otherwise they complete on full.
+  uint64_t* sf_landed = cp_drain + 1;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sf_landed + S);
   volatile int* s_epi_fail = s_abort + 1;
   volatile int* s_last = s_abort + 2;  // stream-K: this pipeline completes the current tile
   int* s_mt = reinterpret_cast<int*>(misc + 1024);
@@ -337,10 +346,11 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_landed[s], 1);
     }
     for (int a = 0; a < ACC; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], C::kEpiWarps);
     }
     mbar_init(drain, 1);
     for (int i = 0; i < C::kSFSlots; ++i) mbar_init(&sf_full[i], C::kSepCp ? C::kCopiers : 1);
@@ -417,28 +427,28 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
         const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
         const int64_t koff = static_cast<int64_t>(kb) * C::kAtomsKT * 512;
+        uint64_t* sf_bar = C::kSepCp ? &sf_landed[st_idx] : &full[st_idx];
         if (side_a) {
+          bulk_load(st + C::kABytes + C::kBBytes, p.sfa + w.sfa_rb * p.sfa_rb_bytes + koff, sf_bytes, sf_bar, pol_a);
           tma_load_2d(st, &tmA, &full[st_idx], kb * 128, w.a_row, pol_a);
-          bulk_load(st + C::kABytes + C::kBBytes, p.sfa + w.sfa_rb * p.sfa_rb_bytes + koff, sf_bytes, &full[st_idx],
-                    pol_a);
         } else {
-          tma_load_2d(st + C::kABytes, &tmB, &full[st_idx], kb * 128, w.b_row, pol_b);
           const int rb0 = w.n0 / 128;
 #pragma unroll
           for (int rb = 0; rb < C::kNRB; ++rb)
             if (rb0 + rb < p.sfb_rbs)
               bulk_load(st + C::kABytes + C::kBBytes + C::kSFABytes + rb * C::kAtomsKT * 512,
-                        p.sfb + w.sfb_off + rb * p.sfb_rb_bytes + koff, sf_bytes, &full[st_idx], pol_b);
+                        p.sfb + w.sfb_off + rb * p.sfb_rb_bytes + koff, sf_bytes, sf_bar, pol_b);
+          tma_load_2d(st + C::kABytes, &tmB, &full[st_idx], kb * 128, w.b_row, pol_b);
         }
       };
-      auto stage_bytes = [&](const Work& w, int kb) -> uint32_t {
+      auto stage_sf_bytes = [&](const Work& w, int kb) -> uint32_t {
         const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
         const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
         const int rb0 = w.n0 / 128;
         int nrb = 0;
 #pragma unroll
         for (int rb = 0; rb < C::kNRB; ++rb) nrb += (rb0 + rb < p.sfb_rbs) ? 1 : 0;
-        return C::kABytes + C::kBBytes + sf_bytes * (1 + nrb);
+        return sf_bytes * (1 + nrb);
       };
       // With an independent operand, the first ring-full of stages loads only that side,
       // then waits for the preceding kernel, then issues the other side of those stages.
@@ -468,7 +478,12 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], stage_bytes(w, kb));
+          if constexpr (C::kSepCp) {
+            mbar_arrive_expect_tx(&sf_landed[stage], stage_sf_bytes(w, kb));
+            mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + stage_sf_bytes(w, kb));
+          }
           if (!replayed) {
             load_side(stage, w, kb, early_a);
             if (++npend == S) replay();
@@ -490,6 +505,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
           if (issued & (1u << s)) {
             volatile int no_abort = 0;
             mbar_wait(&full[s], (issued_par >> s) & 1u, &no_abort);
+            if (C::kSepCp) mbar_wait(&sf_landed[s], (issued_par >> s) & 1u, &no_abort);
           }
       }
     }
@@ -564,11 +580,11 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
-  } else if (C::kSepCp && warp >= 6) {
-    const int cw = warp - 6;  // 0: A's atoms; 1 + rb: B's row-block rb
+  } else if (C::kSepCp && warp >= 2 + C::kEpiWarps) {
+    const int cw = warp - 2 - C::kEpiWarps;  // 0: A's atoms; 1 + rb: B's row-block rb
     if (lane == 0) {
       // ------------------------------------------------------------ scale-factor copier
-      // Stage n's atoms go to TMEM slot n % kSFSlots once the stage has landed and the
+      // Stage n's atoms go to TMEM slot n % kSFSlots once they have landed and the
       // MMAs of stage n - kSFSlots (the slot's previous user) have completed; each slot's
       // copies are committed to sf_full[slot] for the MMA thread.
       Sched<BN> sch(p, s_mt, s_off, vb, vg);
@@ -579,7 +595,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       bool ok = true;
       while (ok && sch.next(w)) {
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, s_abort)) {
+          if (!mbar_wait(&sf_landed[stage], phase, s_abort)) {
             latch_timeout(s_abort, p.status);
             ok = false;
             break;
@@ -621,12 +637,19 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(cp_drain, 0, &no_abort);
     }
-  } else if (warp >= 2 && warp <= 5) {
+  } else if (warp >= 2 && warp < 2 + C::kEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    // a warp reads the TMEM lane quarter given by its warp index in the CTA, modulo 4
+    // a warp reads the TMEM lane quarter given by its warp index in the CTA, modulo 4,
+    // and (with eight epilogue warps) the column half given by its warp index over 4
     const int q = (threadIdx.x >> 5) & 3;
     const int rl = q * 32 + lane;     // accumulator row (TMEM lane) of this thread
-    const int et = lt - 64;           // 0..127
+    const int et = lt - 64;           // 0 .. 32 * kEpiWarps - 1
+    constexpr int CH = C::kEpiCols;
+    const int c0 = ((warp - 2) >> 2) * CH;  // first accumulator column of this thread
+    // BF16 row-major tiles whose columns are all in range are converted into registers
+    // and TMEM is handed back to the MMA thread before the stores, so that they overlap
+    // the next tile's MMAs
+    const bool early_release = C::kSepCp && p.mode != kModeStreamK && p.out_bf16 && !p.transposed && p.vec_store;
     wait_prior_grids();               // the global scales come from earlier kernels
     const float ga = p.ga ? *p.ga : 1.0f;
     Sched<BN> sch(p, s_mt, s_off, vb, vg);
@@ -635,13 +658,13 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
     while (sch.next(w)) {
       const int acc = iter % ACC;
       const uint32_t par = (iter / ACC) & 1;
-      // the four epilogue warps decide together whether to go on, so that none of them
+      // the epilogue warps decide together whether to go on, so that none of them
       // is left behind at a named barrier
       if (et == 0 && !mbar_wait(&acc_full[acc], par, s_abort)) {
         latch_timeout(s_abort, p.status);
         *s_epi_fail = 1;
       }
-      epi_sync(sub);
+      epi_sync(sub, 32 * C::kEpiWarps);
       if (*s_epi_fail) break;
       tc_fence_after();
       const float gb = p.gb ? p.gb[w.group] : 1.0f;
@@ -649,11 +672,33 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       const bool row_ok = rl < w.rows_valid;
       const int row = w.out_row0 + rl;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      if (q * 32 < w.rows_valid) {  // warp-uniform: warps without a valid row skip TMEM
-        // up to 64 columns per TMEM round trip: four loads in flight, one wait
-        constexpr int CW = BN >= 64 ? 64 : BN;
+      bool released = false;
+      if (q * 32 < w.rows_valid && early_release && w.n0 + BN <= p.Nk) {  // warp-uniform
+        uint32_t pk[CH / 2];  // this thread's columns [c0, c0 + CH) as scaled BF16 pairs
+#pragma unroll
+        for (int cw = 0; cw < CH; cw += 16) {
+          uint32_t rr[16];
+          tmem_ld16(taddr + c0 + cw, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; j += 2)
+            pk[(cw + j) / 2] = pack_bf16x2(__uint_as_float(rr[j]) * scale, __uint_as_float(rr[j + 1]) * scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        released = true;
+        if (row_ok) {
+          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.ldo;
+#pragma unroll
+          for (int c = 0; c < CH; c += 8)
+            *reinterpret_cast<uint4*>(orow + w.n0 + c0 + c) = make_uint4(pk[c / 2], pk[c / 2 + 1], pk[c / 2 + 2], pk[c / 2 + 3]);
+        }
+      } else if (q * 32 < w.rows_valid) {  // warp-uniform: warps without a valid row skip TMEM
+        // up to 64 columns per TMEM round trip (32 with eight epilogue warps), one wait
+        constexpr int CW = C::kSepCp ? 32 : CH >= 64 ? 64 : CH;
 #pragma unroll 1
-        for (int cw = 0; cw < BN; cw += CW) {
+        for (int cw = c0; cw < c0 + CH; cw += CW) {
           uint32_t rr[CW / 16][16];
 #pragma unroll
           for (int h = 0; h < CW / 16; ++h) tmem_ld16(taddr + cw + h * 16, rr[h]);
@@ -683,9 +728,11 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
       ++iter;
       if (p.mode == kModeStreamK) {
         // The pipeline whose partial sums complete the tile's K range writes the tile:
@@ -693,19 +740,19 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         // covered to the tile's counter; the one that brings it to num_kb reads the
         // sums back from L2, scales, converts, stores, and clears sums and counter.
         __threadfence();
-        epi_sync(sub);
+        epi_sync(sub, 32 * C::kEpiWarps);
         if (et == 0) {
           __threadfence();
           const int covered = w.kb1 - w.kb0;
           const int before = atomicAdd(p.tile_cnt + w.tile, covered);
           *s_last = before + covered == p.num_kb ? 1 : 0;
         }
-        epi_sync(sub);
+        epi_sync(sub, 32 * C::kEpiWarps);
         if (*s_last) {
           __threadfence();
           if (row_ok) {
             float* src = p.ws + static_cast<int64_t>(row) * p.Nk;
-            for (int c = 0; c < BN; c += 16) {
+            for (int c = c0; c < c0 + CH; c += 16) {
               const int col = w.n0 + c;
               if (col >= p.Nk) break;
               float v[16];
