@@ -6,23 +6,34 @@
 // -> FP32 accumulators -> epilogue; 4.2: the global scale product is fused into the
 // epilogue so no extra pass over memory is needed).
 //
-// Structure (one CTA per SM, persistent; 6 warps):
+// Structure (one CTA per SM, persistent).  128/256-wide tiles, one pipeline per CTA:
 //   warp 0      TMA producer: per 256-wide K step, one 128 x 128-byte box of A, one
-//               BN x 128-byte box of B (both 128-byte swizzled), and the matching
-//               512-byte scale-factor atoms by bulk copy, into a STAGES-deep ring.
-//   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale atoms -> TMEM, replicated to
-//               the 4 sub-partitions) and tcgen05.mma.kind::mxf4nvf4 (NVFP4,
+//               BN x 128-byte box of B (both 128-byte swizzled) on the stage's barrier,
+//               and the matching 512-byte scale-factor atoms (issued first) on a
+//               barrier of their own, into a STAGES-deep ring.
+//   warp 1      TMEM owner; lane 0 issues tcgen05.mma.kind::mxf4nvf4 (NVFP4,
 //               scale_vec::4X, UE4M3) or kind::mxf4 (MXFP4, scale_vec::2X, UE8M0),
 //               M=128, N=BN, K=64 each, accumulating in TMEM; commits free the ring
 //               slot and, at the end of a tile, hand the accumulator to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31), multiply by gA*gB, BF16 (RNE) or FP32 store; with
-//               ACC=2 accumulator buffers the epilogue of tile i overlaps tile i+1.
+//   warps 2..9  epilogue: two warps per TMEM lane quarter (warp w reads lanes
+//               32*(w%4)..+31), one per column half; multiply by gA*gB, BF16 (RNE) or
+//               FP32 stores.  BF16 row-major tiles are packed into registers and the
+//               accumulator is handed back before the stores.
+//   warps 10..  scale-factor copiers (one for A's atoms, one per 128-row block of B's):
+//               tcgen05.cp of a stage's atoms into a TMEM slot, replicated to the four
+//               sub-partitions, while the MMA thread works on earlier stages.
+// 256-wide tiles with M >= 256 run on CTA pairs (clusters of two): the pair computes a
+// 256 x 256 tile with M=256 MMAs (tcgen05 .cta_group::2) issued by the leader; each CTA
+// loads its own 128 rows of A and half of B's rows (so each SM moves a third fewer
+// operand bytes per MMA), all TMA bytes complete on the leader's barriers, and the
+// leader's commits arrive on both CTAs' barriers.
+// Small-N tiles (16..64) run two independent pipelines of 6 warps per CTA, whose MMA
+// thread also issues the scale-factor copies.
 // Schedules: whole tiles (grouped raster for L2 reuse); stream-K over (tile, K-step)
 // units when there are too few tiles to fill the SMs -- each CTA adds its FP32 partial
-// tiles into a workspace with vector reductions and a small finalize kernel applies the
-// global scales, converts, and clears the workspace; grouped MoE tiles enumerated on the
-// device from the expert offsets.
+// tiles into a workspace with vector reductions, and the one whose part completes a
+// tile's K range reads it back, scales, converts, stores and clears it; grouped MoE
+// tiles enumerated on the device from the expert offsets.
 // Decode-sized M (<= 64) runs with the operands swapped: the weight rows fill MMA-M and
 // the few activation rows are MMA-N (16/32/64), which keeps the tensor-core work held per
 // pipeline stage small and therefore many stages of weights in flight.
@@ -95,9 +106,12 @@ struct Sched {
   int64_t total;
 
   int vgrid;         // pipelines in the grid; this one is number vb
+  int mtile;         // output rows per M tile: 128, or 256 for a CTA pair
+  int sub_row;       // CTA pair: this CTA's first row (and first B row) within the tile
   // vb / vg: this pipeline's index among all pipelines of the grid, and their count
-  __device__ Sched(const GemmArgs& args, const int* mt, const int* off, int vb, int vg)
-      : p(args), s_mt(mt), s_off(off), vgrid(vg) {
+  __device__ Sched(const GemmArgs& args, const int* mt, const int* off, int vb, int vg, int mtile_ = 128,
+                   int sub_row_ = 0)
+      : p(args), s_mt(mt), s_off(off), vgrid(vg), mtile(mtile_), sub_row(sub_row_) {
     if (p.mode == kModeStreamK) {
       const int64_t T = p.total_units;
       u = T * vb / vg;
@@ -170,12 +184,12 @@ struct Sched {
   }
 
   __device__ void plain(Work& w, int mt, int nt) {
-    w.a_row = mt * 128;
+    w.a_row = mt * mtile + sub_row;
     w.out_row0 = w.a_row;
-    w.rows_valid = min(128, p.Mk - w.a_row);
+    w.rows_valid = max(0, min(128, p.Mk - w.a_row));
     w.n0 = nt * BN;
-    w.b_row = w.n0;
-    w.sfa_rb = mt;
+    w.b_row = w.n0 + sub_row;  // a pair's CTAs each load half of the tile's B rows
+    w.sfa_rb = w.a_row / 128;
     w.sfb_off = static_cast<int64_t>(w.n0 / 128) * p.sfb_rb_bytes;
     w.group = 0;
   }
@@ -193,8 +207,9 @@ struct Sched {
 template <int BN>
 constexpr int pipes_per_cta() { return BN <= 32 ? FP4_SMALL_N_PIPES : BN <= 64 ? 2 : 1; }
 
-template <int BN, bool MX, int ACC>
+template <int BN, bool MX, int ACC, bool PAIR = false>
 struct Cfg {
+  static_assert(!PAIR || (BN == 256 && ACC == 1), "CTA pairs run 256 x 256 tiles");
   static constexpr int kP = pipes_per_cta<BN>();
   // Single-pipeline kernels (128/256-wide tiles) add copier warps that move each stage's
   // scale factors into TMEM, so that these copies are not serialised behind the MMA
@@ -210,7 +225,7 @@ struct Cfg {
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
-  static constexpr int kBBytes = BN * 128;
+  static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * 128;  // a pair's CTA holds half of B's rows
   static constexpr int kSFABytes = kAtomsKT * 512;
   static constexpr int kSFBBytes = kNRB * kAtomsKT * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // a multiple of 1024
@@ -309,11 +324,12 @@ __device__ __forceinline__ void epi_sync(int sub, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + sub), "r"(nthreads) : "memory");
 }
 
-template <int BN, bool MX, int ACC>
-__global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
+template <int BN, bool MX, int ACC, bool PAIR>
+__global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const GemmArgs p) {
-  using C = Cfg<BN, MX, ACC>;
+  using C = Cfg<BN, MX, ACC, PAIR>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
@@ -339,7 +355,15 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   volatile int* s_last = s_abort + 2;  // stream-K: this pipeline completes the current tile
   int* s_mt = reinterpret_cast<int*>(misc + 1024);
   int* s_off = s_mt + (kMaxGroups + 1);
-  const int vb = blockIdx.x * C::kP + sub, vg = gridDim.x * C::kP;
+  // A CTA pair (cluster of two) shares one 256 x 256 tile: rank 0, the leader, issues the
+  // MMAs and scale-factor copies for both; each CTA loads its own 128 rows of A, its half
+  // of B's rows, its A scales and all of the tile's B scales, and stores its 128 rows.
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int vb = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x) * C::kP + sub;
+  const int vg = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x) * C::kP;
+  constexpr int kMTile = PAIR ? 256 : 128;
+  const int sub_row = static_cast<int>(rank) * 128;
 
   // prologue (overlaps the tail of the previous kernel under programmatic launch)
   if (lt == 0) {
@@ -350,7 +374,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
     }
     for (int a = 0; a < ACC; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], C::kEpiWarps);
+      mbar_init(&acc_empty[a], (PAIR ? 2 : 1) * C::kEpiWarps);  // a pair: both CTAs' epilogue warps
     }
     mbar_init(drain, 1);
     for (int i = 0; i < C::kSFSlots; ++i) mbar_init(&sf_full[i], C::kSepCp ? C::kCopiers : 1);
@@ -363,10 +387,19 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (PAIR) {
+      tma_prefetch_desc(&tmSFA);
+      tma_prefetch_desc(&tmSFB);
+    }
   }
   if (sub == 0 && warp == 1) {  // one allocation for all pipelines of the CTA
-    tmem_alloc(&s_tmem_base, C::kTmemAlloc);
-    tmem_relinquish();
+    if constexpr (PAIR) {       // the same columns in both CTAs of the pair
+      tmem_alloc_pair(&s_tmem_base, C::kTmemAlloc);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&s_tmem_base, C::kTmemAlloc);
+      tmem_relinquish();
+    }
   }
   // the next kernel on the stream may launch now; it waits for this grid to complete
   allow_dependents();
@@ -399,6 +432,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // a pair: the peer's barriers are initialised before this CTA's loads and arrivals reach them
+  if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = s_tmem_base + sub * C::kTmemCols;
   const uint32_t sf_col0 = ACC * BN;
@@ -419,14 +454,35 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       // ------------------------------------------------------------ producer
       // swapped decode: the weights (A here) are read once -> evict first; the small
       // activations (B) are re-read by every CTA -> keep
-      const uint64_t pol_a = p.transposed ? l2_policy_evict_first() : l2_policy_normal();
-      const uint64_t pol_b = p.transposed ? l2_policy_evict_last() : l2_policy_normal();
+      // otherwise both operands are re-read by other tiles -> keep (the output is stored
+      // with the streaming hint, so that it does not push them out of L2)
+      const uint64_t pol_a = p.transposed ? l2_policy_evict_first() : l2_policy_evict_last();
+      const uint64_t pol_b = l2_policy_evict_last();
       // Loads of one stage: the A box and A scales ("a" side), the B box and B scales.
       auto load_side = [&](int st_idx, const Work& w, int kb, bool side_a) {
         uint8_t* st = smem + st_idx * C::kStageBytes;
         const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
         const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
         const int64_t koff = static_cast<int64_t>(kb) * C::kAtomsKT * 512;
+        if constexpr (PAIR) {
+          // every box in full (out-of-range rows read as zero), so that the leader can
+          // expect a fixed byte count from both CTAs on its own barriers
+          const uint32_t c_full = cluster_addr(smem_u32(&full[st_idx]), 0);
+          const uint32_t c_sf = cluster_addr(smem_u32(&sf_landed[st_idx]), 0);
+          if (side_a) {
+            tma_load_2d_pair(st + C::kABytes + C::kBBytes, &tmSFA, c_sf, 0,
+                             static_cast<int>((w.sfa_rb * p.sfa_rb_bytes + koff) / 256), pol_a);
+            tma_load_2d_pair(st, &tmA, c_full, kb * 128, w.a_row, pol_a);
+          } else {
+#pragma unroll
+            for (int rb = 0; rb < C::kNRB; ++rb)
+              tma_load_2d_pair(st + C::kABytes + C::kBBytes + C::kSFABytes + rb * C::kAtomsKT * 512, &tmSFB, c_sf, 0,
+                               static_cast<int>((w.sfb_off + rb * p.sfb_rb_bytes + koff) / 256), pol_b);
+            tma_load_2d_pair(st + C::kABytes, &tmB, c_full, kb * 128, w.b_row, pol_b);
+          }
+          (void)sf_bytes;
+          return;
+        }
         uint64_t* sf_bar = C::kSepCp ? &sf_landed[st_idx] : &full[st_idx];
         if (side_a) {
           bulk_load(st + C::kABytes + C::kBBytes, p.sfa + w.sfa_rb * p.sfa_rb_bytes + koff, sf_bytes, sf_bar, pol_a);
@@ -458,7 +514,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       bool replayed = !early;
       auto replay = [&]() {
         wait_prior_grids();
-        Sched<BN> rs(p, s_mt, s_off, vb, vg);
+        Sched<BN> rs(p, s_mt, s_off, vb, vg, kMTile, sub_row);
         Work rw;
         int j = 0;
         while (j < npend && rs.next(rw))
@@ -466,7 +522,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         replayed = true;
       };
       if (!early) wait_prior_grids();
-      Sched<BN> sch(p, s_mt, s_off, vb, vg);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
       Work w;
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
@@ -478,7 +534,12 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             ok = false;
             break;
           }
-          if constexpr (C::kSepCp) {
+          if constexpr (PAIR) {
+            if (leader) {  // the leader's barriers count the boxes of both CTAs
+              mbar_arrive_expect_tx(&sf_landed[stage], 2 * (C::kSFABytes + C::kSFBBytes));
+              mbar_arrive_expect_tx(&full[stage], 2 * (C::kABytes + C::kBBytes));
+            }
+          } else if constexpr (C::kSepCp) {
             mbar_arrive_expect_tx(&sf_landed[stage], stage_sf_bytes(w, kb));
             mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes);
           } else {
@@ -500,7 +561,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         }
       }
       if (ok && !replayed) replay();
-      if (*s_abort) {  // let every issued copy land before the CTA's shared memory goes away
+      // let every issued copy land before the CTA's shared memory goes away (a pair's
+      // leader waits for both CTAs' boxes: they complete on its barriers)
+      if (*s_abort && leader) {
         for (int s = 0; s < S; ++s)
           if (issued & (1u << s)) {
             volatile int no_abort = 0;
@@ -510,9 +573,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer
-      Sched<BN> sch(p, s_mt, s_off, vb, vg);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
       int stage = 0, iter = 0, nstage = 0;
@@ -555,16 +618,23 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
           for (int k = 0; k < nk; ++k) {
             const uint32_t a_idx = MX ? (k >> 1) : k;
             const uint32_t sfid = MX ? (k & 1) * 2 : 0;
-            const uint32_t idesc = mma_idesc(BN, MX, sfid, sfid);
+            const uint32_t idesc = mma_idesc(BN, MX, sfid, sfid, kMTile);
             const uint32_t accum = (kb > w.kb0 || k > 0) ? 1u : 0u;
             const uint32_t ta = (sfa_t + a_idx * 4) | (sfid << 30);
             const uint32_t tb = (sfb_t + a_idx * C::kNRB * 4) | (sfid << 30);
-            if constexpr (MX)
+            if constexpr (PAIR && MX)
+              tc_mma_mxfp4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
+            else if constexpr (PAIR)
+              tc_mma_nvfp4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
+            else if constexpr (MX)
               tc_mma_mxfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
             else
               tc_mma_nvfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
           }
-          tc_commit(&empty[stage]);
+          if constexpr (PAIR)
+            tc_commit_pair_mc(&empty[stage], 3);  // frees the stage in both CTAs
+          else
+            tc_commit(&empty[stage]);
           if (++slot == C::kSFSlots) slot = 0;
           if (++stage == S) {
             stage = 0;
@@ -572,22 +642,28 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit(&acc_full[acc]);
+        if constexpr (PAIR)
+          tc_commit_pair_mc(&acc_full[acc], 3);  // both CTAs' epilogues
+        else
+          tc_commit(&acc_full[acc]);
         ++iter;
       }
       // make sure no MMA still writes TMEM when it is freed
-      tc_commit(drain);
+      if constexpr (PAIR)
+        tc_commit_pair(drain);
+      else
+        tc_commit(drain);
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
   } else if (C::kSepCp && warp >= 2 + C::kEpiWarps) {
     const int cw = warp - 2 - C::kEpiWarps;  // 0: A's atoms; 1 + rb: B's row-block rb
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------------------ scale-factor copier
       // Stage n's atoms go to TMEM slot n % kSFSlots once they have landed and the
       // MMAs of stage n - kSFSlots (the slot's previous user) have completed; each slot's
       // copies are committed to sf_full[slot] for the MMA thread.
-      Sched<BN> sch(p, s_mt, s_off, vb, vg);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
       int stage = 0, n = 0;
@@ -614,17 +690,25 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
             const uint32_t st = smem_base + stage * C::kStageBytes;
             const uint32_t sfa_t = tmem + sf_col0 + sl * C::kSFSlot;
             const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
+            auto cp = [&](uint32_t taddr, uint64_t sdesc) {
+              if constexpr (PAIR)
+                tc_cp_sf_atom_pair(taddr, sdesc);
+              else
+                tc_cp_sf_atom(taddr, sdesc);
+            };
             if (cw == 0) {
-              for (int a = 0; a < atoms; ++a)
-                tc_cp_sf_atom(sfa_t + a * 4, smem_desc_sf(st + C::kABytes + C::kBBytes + a * 512));
+              for (int a = 0; a < atoms; ++a) cp(sfa_t + a * 4, smem_desc_sf(st + C::kABytes + C::kBBytes + a * 512));
             } else {
               const int rb = cw - 1;
               for (int a = 0; a < atoms; ++a)
-                tc_cp_sf_atom(sfa_t + C::kSFACols + (a * C::kNRB + rb) * 4,
-                              smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
+                cp(sfa_t + C::kSFACols + (a * C::kNRB + rb) * 4,
+                   smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
             }
           }
-          tc_commit(&sf_full[sl]);
+          if constexpr (PAIR)
+            tc_commit_pair(&sf_full[sl]);
+          else
+            tc_commit(&sf_full[sl]);
           ++n;
           if (++stage == S) {
             stage = 0;
@@ -633,7 +717,10 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         }
       }
       // no copy may still write TMEM when it is freed
-      tc_commit(cp_drain);
+      if constexpr (PAIR)
+        tc_commit_pair(cp_drain);
+      else
+        tc_commit(cp_drain);
       volatile int no_abort = 0;
       mbar_wait(cp_drain, 0, &no_abort);
     }
@@ -650,9 +737,16 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
     // and TMEM is handed back to the MMA thread before the stores, so that they overlap
     // the next tile's MMAs
     const bool early_release = C::kSepCp && p.mode != kModeStreamK && p.out_bf16 && !p.transposed && p.vec_store;
+    // hands an accumulator back to the MMA thread (a pair's leader counts both CTAs' warps)
+    auto release_acc = [&](int a) {
+      if constexpr (PAIR)
+        mbar_arrive_cluster(cluster_addr(smem_u32(&acc_empty[a]), 0));
+      else
+        mbar_arrive(&acc_empty[a]);
+    };
     wait_prior_grids();               // the global scales come from earlier kernels
     const float ga = p.ga ? *p.ga : 1.0f;
-    Sched<BN> sch(p, s_mt, s_off, vb, vg);
+    Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
     Work w;
     int iter = 0;
     while (sch.next(w)) {
@@ -686,13 +780,14 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (lane == 0) release_acc(acc);
         released = true;
         if (row_ok) {
           __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.ldo;
 #pragma unroll
-          for (int c = 0; c < CH; c += 8)
-            *reinterpret_cast<uint4*>(orow + w.n0 + c0 + c) = make_uint4(pk[c / 2], pk[c / 2 + 1], pk[c / 2 + 2], pk[c / 2 + 3]);
+          for (int c = 0; c < CH; c += 8)  // streaming stores: the output is not read back here
+            __stcs(reinterpret_cast<uint4*>(orow + w.n0 + c0 + c),
+                   make_uint4(pk[c / 2], pk[c / 2 + 1], pk[c / 2 + 2], pk[c / 2 + 3]));
         }
       } else if (q * 32 < w.rows_valid) {  // warp-uniform: warps without a valid row skip TMEM
         // up to 64 columns per TMEM round trip (32 with eight epilogue warps), one wait
@@ -731,7 +826,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
       if (!released) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (lane == 0) release_acc(acc);
       }
       ++iter;
       if (p.mode == kModeStreamK) {
@@ -786,10 +881,16 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair: neither CTA frees TMEM or leaves (its shared memory is the peer's operand and
+  // barrier target) before both are done
+  if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
   if (sub == 0 && warp == 1) {
     __syncwarp();
-    tmem_dealloc(s_tmem_base, C::kTmemAlloc);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(s_tmem_base, C::kTmemAlloc);
+    else
+      tmem_dealloc(s_tmem_base, C::kTmemAlloc);
   }
 }
 
@@ -862,8 +963,52 @@ bool make_tensor_map_u8(CUtensorMap* m, const void* base, uint64_t inner_bytes, 
   return true;
 }
 
+// A scale-factor buffer as a [bytes / 256, 256] uint8 matrix, boxes of box_rows x 256
+// bytes, no swizzle, rows past the end read as zero: a CTA pair loads a stage's scale
+// atoms with tensor copies (their completion can be counted on the leader's barrier).
+static bool encode_sf_map(CUtensorMap* m, const void* base, uint64_t bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {256, bytes / 256};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool make_sf_map(CUtensorMap* m, const void* base, uint64_t bytes, uint32_t box_rows) {
+  constexpr int kEntries = 16;
+  static MapCacheEntry cache[kEntries];
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const MapCacheEntry& e = cache[i];
+      if (e.base == base && e.inner == 256 && e.rows == bytes / 256 && e.box == box_rows) {
+        *m = e.map;
+        return true;
+      }
+    }
+  }
+  if (!encode_sf_map(m, base, bytes, box_rows)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  MapCacheEntry& e = cache[next];
+  e.base = base;
+  e.inner = 256;
+  e.rows = bytes / 256;
+  e.box = box_rows;
+  e.map = *m;
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  return true;
+}
+
 struct Plan {
   bool swap;
+  bool pair;  // 256 x 256 tiles on CTA pairs
   int BN, ACC, mode;
   int64_t Mk, Nk;
   int tiles_m, tiles_n, num_kb;
@@ -919,6 +1064,13 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
     pl.mode = kModeTile;
     pl.units = tiles;
     pl.ws_bytes = 0;
+    // 256-wide tiles with at least two 128-row blocks: CTA pairs share 256 x 256 tiles,
+    // so that each SM loads a third fewer operand bytes per MMA
+    if (pl.BN == 256 && !pl.swap && M >= 256) {
+      pl.pair = true;
+      pl.tiles_m = static_cast<int>((pl.Mk + 255) / 256);
+      pl.units = static_cast<int64_t>(pl.tiles_m) * pl.tiles_n;
+    }
   }
   return pl;
 }
@@ -933,10 +1085,11 @@ size_t gemm_bf16a_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return (kQuantWorkspaceBytes + 255) / 256 * 256 + gemm_workspace_bytes(M, N, K, 0);
 }
 
-template <int BN, bool MX, int ACC>
-static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int grid, cudaStream_t st) {
-  using C = Cfg<BN, MX, ACC>;
-  auto kern = fp4_gemm_kernel<BN, MX, ACC>;
+template <int BN, bool MX, int ACC, bool PAIR>
+static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
+                       const GemmArgs& a, int64_t units, cudaStream_t st) {
+  using C = Cfg<BN, MX, ACC, PAIR>;
+  auto kern = fp4_gemm_kernel<BN, MX, ACC, PAIR>;
   // the shared-memory opt-in is per device; set it once per (kernel, device)
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -951,32 +1104,52 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
   // and loads of an operand the caller marked as ready) overlaps the previous kernel on
   // the stream; everything else waits for it
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+  int grid = 0;
+  if constexpr (PAIR) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    // persistent: as many pairs as can be resident at once (asked once per device)
+    static int max_pairs[64] = {0};
+    int pairs = (dev >= 0 && dev < 64) ? max_pairs[dev] : 0;
+    if (pairs <= 0) {
+      cfg.gridDim = dim3(2 * static_cast<unsigned>(num_sms() / 2));
+      e = cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      if (pairs <= 0) return cudaErrorInvalidConfiguration;
+      if (dev >= 0 && dev < 64) max_pairs[dev] = pairs;
+    }
+    grid = 2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, pairs)));
+  } else {
+    grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((units + C::kP - 1) / C::kP, num_sms())));
+    if (a.mode == kModeGrouped) grid = num_sms();
+  }
+  cfg.gridDim = dim3(grid);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, a);
 }
 
 template <bool MX>
-static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                            cudaStream_t st) {
+static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                            const CUtensorMap& tsb, const GemmArgs& a, cudaStream_t st) {
   // one CTA per SM at most; a CTA holds pipes_per_cta<BN>() pipelines
-  auto grid_for = [&](int pipes) {
-    if (pl.mode == kModeGrouped) return num_sms();
-    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((pl.units + pipes - 1) / pipes, num_sms())));
-  };
   switch (pl.BN) {
-    case 16: return run<16, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<16>()), st);
-    case 32: return run<32, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<32>()), st);
-    case 64: return run<64, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<64>()), st);
-    case 128: return run<128, MX, 2>(ta, tb, a, grid_for(pipes_per_cta<128>()), st);
-    default: return run<256, MX, 1>(ta, tb, a, grid_for(pipes_per_cta<256>()), st);
+    case 16: return run<16, MX, 2, false>(ta, tb, tsa, tsb, a, pl.units, st);
+    case 32: return run<32, MX, 2, false>(ta, tb, tsa, tsb, a, pl.units, st);
+    case 64: return run<64, MX, 2, false>(ta, tb, tsa, tsb, a, pl.units, st);
+    case 128: return run<128, MX, 2, false>(ta, tb, tsa, tsb, a, pl.units, st);
+    default:
+      return pl.pair ? run<256, MX, 1, true>(ta, tb, tsa, tsb, a, pl.units, st)
+                     : run<256, MX, 1, false>(ta, tb, tsa, tsb, a, pl.units, st);
   }
 }
 
@@ -1017,11 +1190,23 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
     std::swap(kgA, kgB);
     std::swap(rowsA, rowsB);
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tsa, tsb;
   if (!make_tensor_map_u8(&ta, kA, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsA), 128) ||
-      !make_tensor_map_u8(&tb, kB, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsB), static_cast<uint32_t>(pl.BN))) {
+      !make_tensor_map_u8(&tb, kB, static_cast<uint64_t>(g.K / 2), static_cast<uint64_t>(rowsB),
+                          static_cast<uint32_t>(pl.pair ? pl.BN / 2 : pl.BN))) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
     return 1;
+  }
+  tsa = ta;  // unused unless CTA pairs load the scale factors with tensor copies
+  tsb = ta;
+  if (pl.pair) {
+    // one box = one stage's atoms of one 128-row block (4 atoms NVFP4, 2 MXFP4)
+    const uint32_t box_rows = (g.mx ? 2u : 4u) * 512u / 256u;
+    if (!make_sf_map(&tsa, kSA, static_cast<uint64_t>((rowsA + 127) / 128) * atoms_k * 512, box_rows) ||
+        !make_sf_map(&tsb, kSB, static_cast<uint64_t>((rowsB + 127) / 128) * atoms_k * 512, box_rows)) {
+      *why = "cuTensorMapEncodeTiled failed for the scale factors (alignment or driver)";
+      return 1;
+    }
   }
   GemmArgs a{};
   a.sfa = kSA;
@@ -1062,7 +1247,7 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   } else {
     a.sfb_rbs = static_cast<int>((rowsB + 127) / 128);
   }
-  const cudaError_t e = g.mx ? dispatch<true>(pl, ta, tb, a, st) : dispatch<false>(pl, ta, tb, a, st);
+  const cudaError_t e = g.mx ? dispatch<true>(pl, ta, tb, tsa, tsb, a, st) : dispatch<false>(pl, ta, tb, tsa, tsb, a, st);
   if (e != cudaSuccess) {
     *err = e;
     return 2;

@@ -176,6 +176,103 @@ __device__ __forceinline__ void tc_mma_mxfp4(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// A cluster of two CTAs on neighbouring SMs that share one MMA of M = 256 rows: CTA
+// rank 0 (the leader) issues every tcgen05 operation for both; operand tiles, scale
+// factors and accumulators sit at the same shared-memory offsets and TMEM addresses in
+// both CTAs.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of this CTA's shared-memory word `saddr` in the shared memory of cluster CTA
+// `rank` (same offset), as a shared::cluster address.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// All threads of both CTAs; orders shared-memory and barrier state across the pair.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive once on an mbarrier given by its shared::cluster address (possibly the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+}
+
+// 2-D tiled load into this CTA's shared memory whose bytes complete on the mbarrier at
+// shared::cluster address `cbar`, which may be the leader's (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t cbar, int x, int y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cbar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Arrive once on the leader's `bar` when the pair operations issued so far complete.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// The same, arriving on the barrier at `bar`'s offset in every CTA of `mask`.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "h"(mask)
+               : "memory");
+}
+
+// Scale-factor atom copy in both CTAs: each CTA's atom at `sdesc` into its own TMEM.
+__device__ __forceinline__ void tc_cp_sf_atom_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// M = 256 block-scaled MMAs over the pair: A rows 0..127 and B rows 0..N/2-1 from the
+// leader's shared memory, the rest from the peer's; D rows split the same way.
+__device__ __forceinline__ void tc_mma_nvfp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+      "}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_mxfp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+      "}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // 32 lanes x 32-bit, 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -212,16 +309,18 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
 }
 
 // Instruction descriptor of the block-scaled MMA: E2M1 A and B, K-major, FP32
-// accumulation, M = 128, N = n, scale type UE4M3 (mx = false) or UE8M0 (mx = true),
-// sf_id = byte offset of the scale vectors inside the TMEM column.
-__host__ __device__ __forceinline__ uint32_t mma_idesc(int n, bool mx, uint32_t a_sf_id, uint32_t b_sf_id) {
+// accumulation, M = m (128, or 256 over a CTA pair), N = n, scale type UE4M3
+// (mx = false) or UE8M0 (mx = true), sf_id = byte offset of the scale vectors inside
+// the TMEM column.
+__host__ __device__ __forceinline__ uint32_t mma_idesc(int n, bool mx, uint32_t a_sf_id, uint32_t b_sf_id,
+                                                       int m = 128) {
   uint32_t d = 0;
   d |= (b_sf_id & 3u) << 4;
   d |= 1u << 7;                                   // A: E2M1
   d |= 1u << 10;                                  // B: E2M1
   d |= (static_cast<uint32_t>(n) >> 3) << 17;     // N / 8
   d |= (mx ? 1u : 0u) << 23;                      // scale type
-  d |= (128u >> 4) << 24;                         // M / 16
+  d |= (static_cast<uint32_t>(m) >> 4) << 24;     // M / 16
   d |= (a_sf_id & 3u) << 29;
   return d;
 }

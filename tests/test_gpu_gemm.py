@@ -53,10 +53,13 @@ def test_identity_operand_bit_exact(fmt, m, n, k):
 
 
 @pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
-def test_block_scale_placement_bit_exact(fmt):
+@pytest.mark.parametrize("m,n,k", [(256, 256, 512),
+                                   # 160 tiles of 128 x 256: 256 x 256 tiles on CTA pairs
+                                   (2560, 2048, 512)])
+def test_block_scale_placement_bit_exact(fmt, m, n, k):
     """Every block has its own power-of-two scale: pins which scale byte applies to
-    which (row, K-block) on both operands."""
-    m, n, k = 256, 256, 512
+    which (row, K-block) on both operands (on CTA pairs: the second CTA's A rows and
+    scales, and both halves of B's rows and scale row-blocks)."""
     blk = 16 if fmt == fp4.NVFP4 else 32
     rng = np.random.default_rng(7)
     ac = rng.integers(0, 16, (m, k)).astype(np.uint8)
@@ -112,6 +115,11 @@ GEMM_CASES = [
     (32, 200, 8192, fp4.NVFP4, torch.float32),       # decode kernel, N-tile 32, few tiles
     (7, 640, 2080, fp4.NVFP4, torch.bfloat16),       # decode kernel, K tail (2080 = 8*256 + 32)
     (130, 384, 4096, fp4.NVFP4, torch.bfloat16),     # split over K with a ragged M tile
+    # 256 x 256 tiles on CTA pairs (at least 148 tiles of 128 x 256)
+    (4096, 1280, 512, fp4.NVFP4, torch.bfloat16),
+    (2560, 2048, 1024, fp4.MXFP4, torch.float32),    # FP32 out: TMEM handed back after the stores
+    (2432, 2144, 2080, fp4.NVFP4, torch.bfloat16),   # last M tile: second CTA has no rows; last
+                                                     # N tile: 96 columns; K tail of 32
 ]
 
 
