@@ -100,8 +100,9 @@ struct Work {
 template <int BN>
 struct Sched {
   const GemmArgs& p;
-  const int* s_mt;   // grouped: m-tile prefix per group
+  const int* s_mt;   // grouped: 128-row block prefix per group (= A scale row-blocks)
   const int* s_off;  // grouped: row offsets
+  const int* s_pt;   // grouped CTA pairs: 256-row tile prefix per group
   int64_t u, u_end;  // stream-K: current / end unit; tile modes: current unit
   int64_t total;
 
@@ -110,15 +111,15 @@ struct Sched {
   int sub_row;       // CTA pair: this CTA's first row (and first B row) within the tile
   // vb / vg: this pipeline's index among all pipelines of the grid, and their count
   __device__ Sched(const GemmArgs& args, const int* mt, const int* off, int vb, int vg, int mtile_ = 128,
-                   int sub_row_ = 0)
-      : p(args), s_mt(mt), s_off(off), vgrid(vg), mtile(mtile_), sub_row(sub_row_) {
+                   int sub_row_ = 0, const int* pt = nullptr)
+      : p(args), s_mt(mt), s_off(off), s_pt(pt), vgrid(vg), mtile(mtile_), sub_row(sub_row_) {
     if (p.mode == kModeStreamK) {
       const int64_t T = p.total_units;
       u = T * vb / vg;
       u_end = T * (vb + 1) / vg;
       total = T;
     } else if (p.mode == kModeGrouped) {
-      total = static_cast<int64_t>(s_mt[p.num_groups]) * p.tiles_n;
+      total = static_cast<int64_t>(tiles_prefix()[p.num_groups]) * p.tiles_n;
       u = vb;
     } else {
       total = p.total_units;
@@ -146,22 +147,25 @@ struct Sched {
     u += vgrid;
     if (p.mode == kModeGrouped) {
       const int E = p.num_groups;
-      int lo = 0, hi = E - 1;  // last group e with s_mt[e] * tiles_n <= cur
+      const int* tp = tiles_prefix();
+      int lo = 0, hi = E - 1;  // last group e with tp[e] * tiles_n <= cur
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (static_cast<int64_t>(s_mt[mid]) * p.tiles_n <= cur) lo = mid;
+        if (static_cast<int64_t>(tp[mid]) * p.tiles_n <= cur) lo = mid;
         else hi = mid - 1;
       }
       const int e = lo;
-      const int mte = s_mt[e + 1] - s_mt[e];
-      const int64_t local = cur - static_cast<int64_t>(s_mt[e]) * p.tiles_n;
+      const int mte = tp[e + 1] - tp[e];
+      const int64_t local = cur - static_cast<int64_t>(tp[e]) * p.tiles_n;
       const int nt = static_cast<int>(local / mte), mt = static_cast<int>(local % mte);
-      w.a_row = s_off[e] + mt * 128;
+      // a pair's second CTA may get rows of the next group (or none): they are loaded
+      // and multiplied but never stored
+      w.a_row = s_off[e] + mt * mtile + sub_row;
       w.out_row0 = w.a_row;
-      w.rows_valid = min(128, s_off[e + 1] - w.a_row);
+      w.rows_valid = max(0, min(128, s_off[e + 1] - w.a_row));
       w.n0 = nt * BN;
-      w.b_row = e * p.b_rows_per_group + w.n0;
-      w.sfa_rb = s_mt[e] + mt;
+      w.b_row = e * p.b_rows_per_group + w.n0 + sub_row;
+      w.sfa_rb = s_mt[e] + mt * (mtile / 128) + sub_row / 128;
       w.sfb_off = e * p.sfb_group_bytes + static_cast<int64_t>(w.n0 / 128) * p.sfb_rb_bytes;
       w.group = e;
       w.kb0 = 0;
@@ -182,6 +186,9 @@ struct Sched {
     w.tile = static_cast<int>(cur);
     return true;
   }
+
+  // grouped: M-tile prefix per group in this schedule's tile height
+  __device__ const int* tiles_prefix() const { return mtile == 256 ? s_pt : s_mt; }
 
   __device__ void plain(Work& w, int mt, int nt) {
     w.a_row = mt * mtile + sub_row;
@@ -230,7 +237,7 @@ struct Cfg {
   static constexpr int kSFBBytes = kNRB * kAtomsKT * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // a multiple of 1024
   // grouped schedules use 128-wide tiles only, so multi-pipeline kernels skip the group tables
-  static constexpr int kGroupBytes = kP == 1 ? 2 * (kMaxGroups + 1) * 4 : 0;
+  static constexpr int kGroupBytes = kP == 1 ? (PAIR ? 3 : 2) * (kMaxGroups + 1) * 4 : 0;
   static constexpr int kMiscBytes = 1024 /*barriers, flags*/ + kGroupBytes;
   // the opt-in limit per block, less the alignment slack and the static shared memory
   static constexpr int kSmemLimit = 227 * 1024 - 1024 - 256;
@@ -355,6 +362,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
   volatile int* s_last = s_abort + 2;  // stream-K: this pipeline completes the current tile
   int* s_mt = reinterpret_cast<int*>(misc + 1024);
   int* s_off = s_mt + (kMaxGroups + 1);
+  int* s_pt = PAIR ? s_off + (kMaxGroups + 1) : nullptr;
   // A CTA pair (cluster of two) shares one 256 x 256 tile: rank 0, the leader, issues the
   // MMAs and scale-factor copies for both; each CTA loads its own 128 rows of A, its half
   // of B's rows, its A scales and all of the tile's B scales, and stores its 128 rows.
@@ -407,26 +415,37 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
     wait_prior_grids();  // the offsets may come from the previous kernel
     // m-tile prefix per group (= scale row-block prefix of the grouped A layout)
     const int E = p.num_groups;
-    int carry = 0;
+    // (CTA pairs: also the prefix of 256-row tiles, by which they enumerate tiles)
+    int carry = 0, carry2 = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane;
-      int cnt = 0;
+      int cnt = 0, cnt2 = 0;
       if (e < E) {
         const int lo = p.offsets[e], hi = p.offsets[e + 1];
         s_off[e] = lo;
         cnt = (hi - lo + 127) / 128;
+        cnt2 = (hi - lo + 255) / 256;
       }
-      int incl = cnt;
+      int incl = cnt, incl2 = cnt2;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += t;
+        const int t2 = __shfl_up_sync(0xFFFFFFFFu, incl2, d);
+        if (lane >= d) {
+          incl += t;
+          incl2 += t2;
+        }
       }
-      if (e < E) s_mt[e] = carry + incl - cnt;
+      if (e < E) {
+        s_mt[e] = carry + incl - cnt;
+        if (PAIR) s_pt[e] = carry2 + incl2 - cnt2;
+      }
       carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      carry2 += __shfl_sync(0xFFFFFFFFu, incl2, 31);
     }
     if (lane == 0) {
       s_mt[E] = carry;
+      if (PAIR) s_pt[E] = carry2;
       s_off[E] = p.offsets[E];
     }
   }
@@ -514,7 +533,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
       bool replayed = !early;
       auto replay = [&]() {
         wait_prior_grids();
-        Sched<BN> rs(p, s_mt, s_off, vb, vg, kMTile, sub_row);
+        Sched<BN> rs(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
         Work rw;
         int j = 0;
         while (j < npend && rs.next(rw))
@@ -522,7 +541,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
         replayed = true;
       };
       if (!early) wait_prior_grids();
-      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
       Work w;
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
@@ -575,7 +594,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer
-      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
       int stage = 0, iter = 0, nstage = 0;
@@ -663,7 +682,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
       // Stage n's atoms go to TMEM slot n % kSFSlots once they have landed and the
       // MMAs of stage n - kSFSlots (the slot's previous user) have completed; each slot's
       // copies are committed to sf_full[slot] for the MMA thread.
-      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
+      Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
       const uint32_t smem_base = smem_u32(smem);
       Work w;
       int stage = 0, n = 0;
@@ -746,7 +765,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
     };
     wait_prior_grids();               // the global scales come from earlier kernels
     const float ga = p.ga ? *p.ga : 1.0f;
-    Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row);
+    Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
     Work w;
     int iter = 0;
     while (sch.next(w)) {
@@ -1027,6 +1046,7 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
     pl.swap = false;
     pl.BN = N >= 256 ? 256 : 128;
     pl.ACC = pl.BN == 256 ? 1 : 2;
+    pl.pair = pl.BN == 256;  // 256 x 256 tiles (per expert) on CTA pairs
     pl.mode = kModeGrouped;
     pl.Mk = M;
     pl.Nk = N;
@@ -1129,7 +1149,8 @@ static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
       if (pairs <= 0) return cudaErrorInvalidConfiguration;
       if (dev >= 0 && dev < 64) max_pairs[dev] = pairs;
     }
-    grid = 2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, pairs)));
+    // (grouped schedules count their tiles on the device: every pair)
+    grid = 2 * static_cast<int>(a.mode == kModeGrouped ? pairs : std::max<int64_t>(1, std::min<int64_t>(units, pairs)));
   } else {
     grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((units + C::kP - 1) / C::kP, num_sms())));
     if (a.mode == kModeGrouped) grid = num_sms();
@@ -1202,7 +1223,10 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   if (pl.pair) {
     // one box = one stage's atoms of one 128-row block (4 atoms NVFP4, 2 MXFP4)
     const uint32_t box_rows = (g.mx ? 2u : 4u) * 512u / 256u;
-    if (!make_sf_map(&tsa, kSA, static_cast<uint64_t>((rowsA + 127) / 128) * atoms_k * 512, box_rows) ||
+    // grouped A scales: the capacity fp4_scales_bytes_grouped gives (every 128-row block
+    // of every group plus one pad block per group), which the caller's buffer holds
+    const int64_t sfa_blocks = (rowsA + 127) / 128 + (grouped ? g.num_groups : 0);
+    if (!make_sf_map(&tsa, kSA, static_cast<uint64_t>(sfa_blocks) * atoms_k * 512, box_rows) ||
         !make_sf_map(&tsb, kSB, static_cast<uint64_t>((rowsB + 127) / 128) * atoms_k * 512, box_rows)) {
       *why = "cuTensorMapEncodeTiled failed for the scale factors (alignment or driver)";
       return 1;

@@ -201,7 +201,8 @@ fp4_status fp4_gemm_noalloc(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA
  * MXFP4): for each group e, rows [offsets[e], offsets[e+1]) of A times expert e's
  * weights B_dev + e*N*K/2 give the same rows of D:
  *   D[r, n] = gA * gB[e] * sum_k ...   (as fp4_gemm).
- *   A_dev [total_rows, K/2] with grouped scales sA_dev (fp4_quantize_grouped);
+ *   A_dev [total_rows, K/2] with grouped scales sA_dev (fp4_quantize_grouped; the
+ *   buffer holds fp4_scales_bytes_grouped(total_rows, num_groups, K, fmt) bytes);
  *   B_dev [num_groups, N, K/2], sB_dev num_groups consecutive fp4_scales_bytes(N, K)
  *   blocks; gB_dev [num_groups] floats or NULL; offsets_dev device int32 [groups+1]
  *   with offsets[num_groups] == total_rows.  D_dev [total_rows, N].
