@@ -405,7 +405,7 @@ def run_prefill(args, dev):
     return _line("prefill-shaped NVFP4 GEMM M=N=K=8192, bf16 activations quantized every step, bf16 out",
                  step_tf, "TFLOP/s", step_ms, args, {
                      "dtype": "nvfp4 x nvfp4 -> fp32 accumulate, bf16 out",
-                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1>",
+                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1, CTA pair>",
                                   "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tf / peak,
                                   "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)",
                                   "frac_of_nominal_9pf": gemm_tf / 9000.0, "launch_ms": gemm_ms,
@@ -460,7 +460,7 @@ def run_moe(args, dev):
                  flop / (step_ms * 1e-3) / 1e12, "TFLOP/s", step_ms, args, {
                      "dtype": "mxfp4 x mxfp4 -> fp32 accumulate, bf16 out",
                      "roofline": {"bound": "tensor" if flop / peak > gemm_bytes / hbm * 1e-3 else "hbm",
-                                  "kernel": "fp4_gemm_kernel<128, mxfp4, 2> (grouped)",
+                                  "kernel": "fp4_gemm_kernel<256, mxfp4, 1, CTA pair> (grouped)",
                                   "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
                                   "frac": t_roof / gemm_ms,
                                   "frac_definition": "roofline time (slower of tensor and HBM) / measured time",
@@ -517,7 +517,7 @@ def run_train(args, dev):
                  "per step, forward X W^T and backward dY W, bf16 out", big["step_TFLOP/s"], "TFLOP/s",
                  big["step_ms"], args, {
                      "dtype": "nvfp4 x nvfp4 -> fp32 accumulate, bf16 out",
-                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1> at S=16384",
+                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1, CTA pair> at S=16384",
                                   "achieved": big["fwd_TFLOP/s"], "peak": peak, "unit": "TFLOP/s",
                                   "frac": big["fwd_frac"], "traffic": None,
                                   "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g}"},
