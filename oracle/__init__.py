@@ -16,6 +16,12 @@ scale factors re-applied to the FP32 accumulators; "FP4" glossary entry
 "MXFP4 / NVFP4 video transcript" (prism.simon-ai.net) -- NVFP4's FP32 tensor scale,
 16x16 weight blocks.
 
+The next steps after the hot path have their definitions here too, ahead of any
+kernel: the epilogue's bias and activation ("Rubin FP4 GEMM overview" 3.2 and 4.2),
+the random Hadamard transform and stochastic rounding of the NVFP4 training recipe
+("MXFP4 / NVFP4 video transcript", training-recipe passage; "FP4" glossary entry,
+section "Inference and training in FP4").
+
 Parity pins: every function here is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_*.py`` (code enumeration, library conversions, the glossary's
 printed block-size experiment, hand-worked blocks, invariants, exact-rational brute
@@ -72,6 +78,9 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_amax": (I32, [P, I64, I32, P]),
         "orc_global_scale": (ctypes.c_float, [ctypes.c_float]),
         "orc_quantize_nvfp4_1d": (I32, [P, I64, I64, I32, P, P, P, P]),
+        "orc_quantize_nvfp4_1d_r": (I32, [P, I64, I64, I32, P, P, P, P, P]),
+        "orc_e2m1_encode_sr": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_uint32]),
+        "orc_rht16": (I32, [P, I64, I64, I32, ctypes.c_uint32, P]),
         "orc_quantize_mxfp4_1d": (I32, [P, I64, I64, I32, P, P]),
         "orc_quantize_nvfp4_2d": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
         "orc_scales_bytes": (I64, [I64, I64]),
@@ -310,3 +319,84 @@ def bf16_ulp(v: np.ndarray) -> np.ndarray:
         e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
     e = np.maximum(e, -126.0)
     return np.ldexp(1.0, (e - 7).astype(np.int64))
+
+
+# ---------------------------------------------------------------- next steps
+def epilogue(d: np.ndarray, bias=None, act: str = "none") -> np.ndarray:
+    """The epilogue after the scale factors ("Rubin FP4 GEMM overview" 3.2: the FP32
+    result is multiplied by the scale factors, the bias is added, the activation is
+    applied, then it is converted to the output format; 4.2: C = (A.B)(sA.sB) + bias).
+    ``d`` is the scaled product (``gemm_reference`` of the dequantized operands);
+    ``bias`` [N] is added to every row; ``act`` is "none" or "relu" (the pages name no
+    activation; ReLU is the plainest).  FP64."""
+    out = np.asarray(d, dtype=np.float64)
+    if bias is not None:
+        out = out + np.asarray(bias, dtype=np.float64)[None, :]
+    if act == "relu":
+        out = np.maximum(out, 0.0)
+    elif act != "none":
+        raise ValueError(f"unknown activation {act}")
+    return out
+
+
+def hadamard16() -> np.ndarray:
+    """The 16x16 Sylvester Hadamard matrix by its definition, H[i, j] =
+    (-1)^popcount(i & j)."""
+    i = np.arange(16)[:, None]
+    j = np.arange(16)[None, :]
+    return np.where(np.vectorize(lambda v: bin(v).count("1") % 2)(i & j) == 1, -1.0, 1.0)
+
+
+def rht16_reference(x: np.ndarray, signs: int) -> np.ndarray:
+    """Random Hadamard transform, FP64 definition: each 16-element block b of a row
+    becomes Q b with Q = (1/4) H16 diag(s), s_i = -1 where bit i of ``signs`` is set
+    ("MXFP4 / NVFP4 video transcript", training-recipe passage: the values are mixed,
+    the vector's magnitude is kept, a dot product of two transformed operands is
+    unchanged)."""
+    x = np.asarray(x, dtype=np.float64)
+    rows, cols = x.shape
+    s = np.array([-1.0 if (signs >> i) & 1 else 1.0 for i in range(16)])
+    q = hadamard16() * s[None, :] / 4.0
+    return (x.reshape(rows, cols // 16, 16) @ q.T).reshape(rows, cols)
+
+
+def rht16(x: np.ndarray, signs: int) -> np.ndarray:
+    """The same transform in FP32, in the fast Walsh-Hadamard order (the signs, the
+    butterfly stages of half-width 1, 2, 4, 8, then the factor 1/4): the order a kernel
+    uses, so that both sides quantize the same FP32 values."""
+    xa, dt = _as_input(x)
+    if xa.ndim == 1:
+        xa = xa.reshape(1, -1)
+    rows, cols = xa.shape
+    out = np.zeros((rows, cols), np.float32)
+    if _L().orc_rht16(_ptr(xa), rows, cols, dt, ctypes.c_uint32(signs & 0xFFFF), _ptr(out)) != 0:
+        raise NonFiniteInput("non-finite element")
+    return out
+
+
+def e2m1_encode_sr(v: float, bits: int) -> int:
+    """Stochastic E2M1 rounding of one FP32 value with one 32-bit random word."""
+    return int(_L().orc_e2m1_encode_sr(ctypes.c_float(v), ctypes.c_uint32(bits)))
+
+
+def quantize_sr(x: np.ndarray, rbits: np.ndarray, g_in=None):
+    """NVFP4 1-D quantize with stochastic rounding of the elements (the block scales
+    are the round-to-nearest quantizer's; "MXFP4 / NVFP4 video transcript",
+    training-recipe passage, fourth part).  ``rbits``: one uint32 per element, the
+    random numbers the method draws, passed in.  Returns codes / scales / g as
+    ``quantize``."""
+    xa, dt = _as_input(x)
+    if xa.ndim == 1:
+        xa = xa.reshape(1, -1)
+    rows, cols = xa.shape
+    rb = np.ascontiguousarray(rbits, dtype=np.uint32).reshape(rows, cols)
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    sc = np.zeros((rows, cols // 16), np.uint8)
+    gbuf = np.zeros(1, np.float32)
+    gin = None if g_in is None else np.array([g_in], np.float32)
+    rc = _L().orc_quantize_nvfp4_1d_r(_ptr(xa), rows, cols, dt, _ptr(gin) if gin is not None else None, _ptr(rb),
+                                      _ptr(codes), _ptr(sc), _ptr(gbuf))
+    if rc != 0:
+        raise NonFiniteInput("non-finite element")
+    return {"codes": codes, "scales": sc, "g": np.float32(gbuf[0])}
+

@@ -39,6 +39,14 @@
  *    zero element gives a zero code even if the reciprocal overflowed.
  *  - Packing: two codes per byte, the even element in the low nibble.
  *  - Scale-factor layout: 128x4 atoms of 512 bytes (see orc_swizzle_scales).
+ *  - Stochastic rounding ([P2] training-recipe passage, its fourth part): only the
+ *    element rounding changes; the block scale is the deterministic one.  u is a
+ *    24-bit uniform in [0, 1) taken from caller-supplied random bits.
+ *  - Random Hadamard transform ([P2] training-recipe passage, its third part; [P4]
+ *    section "Inference and training in FP4"): 16-element blocks along the rows,
+ *    y = (1/4) H16 diag(s) x with the Sylvester H16 and one caller-supplied sign
+ *    vector s; in FP32 the four butterfly stages of the fast Walsh-Hadamard
+ *    transform, in order.
  */
 #include <math.h>
 #include <stdint.h>
@@ -119,6 +127,29 @@ uint8_t orc_e2m1_encode(float v) {
         }
     }
     return (uint8_t)(best | sign);
+}
+
+/* Stochastic rounding ([P2] training-recipe passage, fourth part: 0.3 between the
+ * representable 0 and 1 becomes 1 with probability 0.3 and 0 otherwise, so that the
+ * expected value is the value).  |v| between the neighbouring magnitudes lo < |v| < hi
+ * goes to hi iff u < (|v| - lo) / (hi - lo), with u = (bits >> 8) * 2^-24 in [0, 1);
+ * magnitudes on the grid are kept, magnitudes at or beyond 6 saturate to 6.  Both the
+ * difference and the division are exact in FP32 (lo <= |v| < hi <= 2 lo or lo = 0,
+ * and the gap is a power of two), so the decision does not depend on the precision.
+ * The sign bit copies v's sign. */
+uint8_t orc_e2m1_encode_sr(float v, uint32_t bits) {
+    uint8_t sign = signbit(v) ? 8 : 0;
+    float a = fabsf(v);
+    if (a >= 6.0f) return (uint8_t)(7 | sign);
+    int lo = 0;  /* the largest magnitude not above a */
+    for (int c = 1; c < 8; ++c)
+        if (e2m1_magnitude(c) <= (double)a) lo = c;
+    float lov = (float)e2m1_magnitude(lo);
+    if (a == lov) return (uint8_t)(lo | sign);
+    float gap = (float)e2m1_magnitude(lo + 1) - lov;
+    float frac = (a - lov) / gap;
+    float u = (float)(bits >> 8) * 0x1p-24f;
+    return (uint8_t)((u < frac ? lo + 1 : lo) | sign);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -233,8 +264,10 @@ float orc_global_scale(float amax_t) {
 /* ------------------------------------------------------------------------- */
 
 /* Encodes n values xs[] with block amax amax_b and global scale g; returns the
- * scale byte and writes the n 4-bit codes. */
-static uint8_t nvfp4_encode_block(const float* xs, int n, float amax_b, float g, uint8_t* codes) {
+ * scale byte and writes the n 4-bit codes (rounded to nearest, or stochastically
+ * with one 32-bit random word per element when rbits is not NULL). */
+static uint8_t nvfp4_encode_block(const float* xs, int n, float amax_b, float g, const uint32_t* rbits,
+                                  uint8_t* codes) {
     float t = amax_b / 6.0f;
     float r = t / g;
     uint8_t sb = orc_e4m3_encode(r);
@@ -247,7 +280,9 @@ static uint8_t nvfp4_encode_block(const float* xs, int n, float amax_b, float g,
     /* A zero element encodes as a zero code even when 1/denom overflowed to inf
      * (a denominator below 2^-128): the ratio x / denom of a zero is zero. */
     for (int i = 0; i < n; ++i)
-        codes[i] = xs[i] == 0.0f ? (signbit(xs[i]) ? 8 : 0) : orc_e2m1_encode(xs[i] * inv);
+        codes[i] = xs[i] == 0.0f   ? (signbit(xs[i]) ? 8 : 0)
+                   : rbits != NULL ? orc_e2m1_encode_sr(xs[i] * inv, rbits[i])
+                                   : orc_e2m1_encode(xs[i] * inv);
     return sb;
 }
 
@@ -277,8 +312,10 @@ static void pack_row(const uint8_t* codes, int64_t n, uint8_t* out) {
 /* g_in: caller's global scale (NVFP4), or NULL to compute amax first.         */
 /* ------------------------------------------------------------------------- */
 
-int orc_quantize_nvfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
-                          const float* g_in, uint8_t* codes, uint8_t* scales_rm, float* g_out) {
+/* rbits: NULL (round to nearest) or one random word per element, row-major
+ * [rows, cols], for stochastic rounding. */
+int orc_quantize_nvfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype, const float* g_in,
+                            const uint32_t* rbits, uint8_t* codes, uint8_t* scales_rm, float* g_out) {
     /* a non-finite element is an error whether or not the caller supplies g */
     float amax_t, g;
     if (orc_amax(x, rows * cols, dtype, &amax_t) != ORC_OK) return ORC_ERR_NONFINITE;
@@ -294,13 +331,19 @@ int orc_quantize_nvfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
                 xs[i] = load_elem(x, r * cols + b * 16 + i, dtype);
                 if (fabsf(xs[i]) > amax_b) amax_b = fabsf(xs[i]);
             }
-            scales_rm[r * (cols / 16) + b] = nvfp4_encode_block(xs, 16, amax_b, g, cb);
+            scales_rm[r * (cols / 16) + b] =
+                nvfp4_encode_block(xs, 16, amax_b, g, rbits ? rbits + r * cols + b * 16 : NULL, cb);
             memcpy(row_codes + b * 16, cb, 16);
         }
         pack_row(row_codes, cols, codes + r * (cols / 2));
     }
     free(row_codes);
     return ORC_OK;
+}
+
+int orc_quantize_nvfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
+                          const float* g_in, uint8_t* codes, uint8_t* scales_rm, float* g_out) {
+    return orc_quantize_nvfp4_1d_r(x, rows, cols, dtype, g_in, NULL, codes, scales_rm, g_out);
 }
 
 int orc_quantize_mxfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
@@ -352,7 +395,7 @@ int orc_quantize_nvfp4_2d(const void* x, int64_t rows, int64_t cols, int dtype, 
                     xs[i * 16 + j] = v;
                     if (fabsf(v) > amax_b) amax_b = fabsf(v);
                 }
-            uint8_t sb = nvfp4_encode_block(xs, 256, amax_b, g, cb);
+            uint8_t sb = nvfp4_encode_block(xs, 256, amax_b, g, NULL, cb);
             for (int i = 0; i < 16; ++i) {
                 for (int j = 0; j < 16; ++j) full[(tr * 16 + i) * cols + tc * 16 + j] = cb[i * 16 + j];
                 scales_rm[(tr * 16 + i) * (cols / 16) + tc] = sb;       /* row of W    */
@@ -465,6 +508,38 @@ void orc_fake_quant_fp32_scale(const float* x, int64_t n, int64_t block, float* 
             deq[b * block + i] = mag * sgn * scale;
         }
     }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Random Hadamard transform ([P2] training-recipe passage, third part: the values */
+/* of a block are mixed so that an outlier no longer sets the block scale alone;   */
+/* the vector's magnitude is unchanged, and so is a dot product when both operands */
+/* are transformed alike).  Each 16-element block b of a row becomes               */
+/* (1/4) H16 diag(s) b, s_i = -1 where bit i of `signs` is set, H16 the Sylvester  */
+/* Hadamard matrix.  FP32, in the order of the fast Walsh-Hadamard transform: the  */
+/* signs, then butterfly stages with half-widths 1, 2, 4, 8 (pairs j, j + h become */
+/* their sum and difference), then the exact factor 1/4.  cols % 16 == 0.          */
+/* ------------------------------------------------------------------------- */
+
+int orc_rht16(const void* x, int64_t rows, int64_t cols, int dtype, uint32_t signs, float* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            float v[16];
+            for (int i = 0; i < 16; ++i) {
+                v[i] = load_elem(x, r * cols + b * 16 + i, dtype);
+                if (!isfinite(v[i])) return ORC_ERR_NONFINITE;
+                if ((signs >> i) & 1u) v[i] = -v[i];
+            }
+            for (int h = 1; h < 16; h *= 2)
+                for (int i = 0; i < 16; i += 2 * h)
+                    for (int j = i; j < i + h; ++j) {
+                        float p = v[j], q = v[j + h];
+                        v[j] = p + q;
+                        v[j + h] = p - q;
+                    }
+            for (int i = 0; i < 16; ++i) out[r * cols + b * 16 + i] = v[i] * 0.25f;
+        }
+    return ORC_OK;
 }
 
 /* ------------------------------------------------------------------------- */

@@ -13,6 +13,7 @@ import pytest
 import oracle
 import test_oracle_formats as tf
 import test_oracle_gemm as tg
+import test_oracle_next as tn
 import test_oracle_quantize as tq
 
 with open(oracle._SRC) as _f:
@@ -98,6 +99,36 @@ C_MUTATIONS = [
      "float scale = amax_b / 6.0f;",
      "float scale = amax_b / 5.0f;",
      [tq.test_glossary_block_size_experiment_exact]),
+    # stochastic rounding and the Hadamard transform (the steps after the hot path)
+    ("stochastic rounding goes up when u equals the fraction",
+     "return (uint8_t)((u < frac ? lo + 1 : lo) | sign);",
+     "return (uint8_t)((u <= frac ? lo + 1 : lo) | sign);",
+     [lambda: tn.test_sr_expectation_over_a_uniform_grid_of_u(0.75),
+      lambda: tn.test_sr_expectation_over_a_uniform_grid_of_u(1.25)]),
+    ("stochastic rounding goes up with probability 1 - fraction",
+     "return (uint8_t)((u < frac ? lo + 1 : lo) | sign);",
+     "return (uint8_t)((u >= frac ? lo + 1 : lo) | sign);",
+     [lambda: tn.test_sr_expectation_over_a_uniform_grid_of_u(0.3), tn.test_quantize_sr_keeps_the_block_scales_and_is_unbiased]),
+    ("stochastic quantize rounds to nearest",
+     "rbits != NULL ? orc_e2m1_encode_sr(xs[i] * inv, rbits[i])",
+     "rbits != NULL ? orc_e2m1_encode(xs[i] * inv)",
+     [tn.test_quantize_sr_keeps_the_block_scales_and_is_unbiased, tn.test_quantize_sr_with_zero_bits_rounds_every_magnitude_up]),
+    ("Hadamard butterfly skips the first stage",
+     "for (int h = 1; h < 16; h *= 2)",
+     "for (int h = 2; h < 16; h *= 2)",
+     [lambda: tn.test_rht_spreads_a_spike_evenly(0x0000, 5), tn.test_rht_fp32_within_the_butterfly_bound]),
+    ("Hadamard transform without the factor 1/4",
+     "out[r * cols + b * 16 + i] = v[i] * 0.25f;",
+     "out[r * cols + b * 16 + i] = v[i];",
+     [lambda: tn.test_rht_spreads_a_spike_evenly(0x0000, 0), tn.test_rht_fp32_within_the_butterfly_bound]),
+    ("Hadamard signs read from the high bit down",
+     "if ((signs >> i) & 1u) v[i] = -v[i];",
+     "if ((signs >> (15 - i)) & 1u) v[i] = -v[i];",
+     [lambda: tn.test_rht_spreads_a_spike_evenly(0x00FF, 0), tn.test_rht_fp32_within_the_butterfly_bound]),
+    ("Hadamard butterfly difference reversed",
+     "v[j + h] = p - q;",
+     "v[j + h] = q - p;",
+     [lambda: tn.test_rht_spreads_a_spike_evenly(0x0000, 5), tn.test_rht_fp32_within_the_butterfly_bound]),
 ]
 
 
@@ -162,3 +193,49 @@ def _ulp_one_bit_short(v):
 def test_planted_python_mistake_is_caught(monkeypatch, attr, wrong, pins):
     monkeypatch.setattr(oracle, attr, wrong)
     assert _caught(pins) > 0
+
+
+# Python-level steps of the Hadamard transform's definition and of the epilogue
+_H = oracle.hadamard16()
+
+
+def _hadamard_sequency_order():
+    """The rows sorted by their number of sign changes (Walsh order), a common slip."""
+    changes = (np.diff(_H, axis=1) != 0).sum(1)
+    return _H[np.argsort(changes, kind="stable")]
+
+
+def _rht_norm_sixteenth(x, signs):
+    return oracle_rht_reference(x, signs) / 4.0
+
+
+def _rht_signs_on_rows(x, signs):
+    x = np.asarray(x, dtype=np.float64)
+    rows, cols = x.shape
+    s = np.array([-1.0 if (signs >> i) & 1 else 1.0 for i in range(16)])
+    q = s[:, None] * _H / 4.0
+    return (x.reshape(rows, cols // 16, 16) @ q.T).reshape(rows, cols)
+
+
+def _epilogue_relu_before_bias(d, bias=None, act="none"):
+    out = np.asarray(d, dtype=np.float64)
+    if act == "relu":
+        out = np.maximum(out, 0.0)
+    if bias is not None:
+        out = out + np.asarray(bias, dtype=np.float64)[None, :]
+    return out
+
+
+oracle_rht_reference = oracle.rht16_reference
+
+
+@pytest.mark.parametrize("attr,wrong,pins", [
+    ("hadamard16", _hadamard_sequency_order, [tn.test_hadamard16_matches_scipy]),
+    ("rht16_reference", _rht_norm_sixteenth, [tn.test_rht_keeps_block_norms, lambda: tn.test_rht_is_orthonormal(0x1234)]),
+    ("rht16_reference", _rht_signs_on_rows, [lambda: tn.test_rht_spreads_a_spike_evenly(0x00FF, 0)]),
+    ("epilogue", _epilogue_relu_before_bias, [tn.test_epilogue_order_scale_bias_activation]),
+])
+def test_planted_python_mistake_in_the_next_steps_is_caught(monkeypatch, attr, wrong, pins):
+    monkeypatch.setattr(oracle, attr, wrong)
+    assert _caught(pins) > 0
+
