@@ -154,8 +154,9 @@ def decode_bytes(m: int, n: int, k: int):
 
 
 def traffic_for(kernel_key: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if the library has not
-    changed since it was taken (else None)."""
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel's sources (the
+    entry's "sources", else the whole library) have not changed since it was taken
+    (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -164,7 +165,11 @@ def traffic_for(kernel_key: str):
             t = json.load(f)
         from block_scaled_fp4_04_b200 import build as fp4_build
         entry = t.get(kernel_key)
-        if not entry or entry.get("fingerprint") != fp4_build._fingerprint():
+        if not entry:
+            return None
+        srcs = entry.get("sources")
+        fp = fp4_build.sources_fingerprint(srcs) if srcs else fp4_build._fingerprint()
+        if entry.get("fingerprint") != fp:
             return None
         return entry.get("dram_bytes_per_launch")
     except Exception:

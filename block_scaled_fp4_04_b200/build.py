@@ -33,13 +33,32 @@ def _sources():
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
+def _flags_id(extra=()) -> str:
+    """The build flags as text, without the checkout's location: the same tree builds
+    the same library wherever it sits (a GPU machine runs it from a scratch path)."""
+    inc = f"-I{os.path.join(ROOT, 'include')}"
+    return " ".join("-I<repo>/include" if f == inc else f for f in ARCH + FLAGS + list(extra))
+
+
 def _fingerprint(extra=()) -> str:
     h = hashlib.sha256()
     for d in (CSRC, os.path.join(ROOT, "include")):
         for f in sorted(os.listdir(d)):
             with open(os.path.join(d, f), "rb") as fh:
                 h.update(f.encode() + fh.read())
-    h.update(" ".join(ARCH + FLAGS + list(extra)).encode())
+    h.update(_flags_id(extra).encode())
+    return h.hexdigest()
+
+
+def sources_fingerprint(rel_paths, extra=()) -> str:
+    """Fingerprint of one kernel's translation unit: the named files (paths relative to
+    the package directory, e.g. "csrc/fp4_decode.cu") and the build flags.  Profiler
+    counters recorded for that kernel stay valid while it is unchanged."""
+    h = hashlib.sha256()
+    for rel in sorted(rel_paths):
+        with open(os.path.join(PKG, rel), "rb") as fh:
+            h.update(rel.encode() + fh.read())
+    h.update(_flags_id(extra).encode())
     return h.hexdigest()
 
 

@@ -352,9 +352,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
   uint64_t* acc_empty = acc_full + ACC;
   uint64_t* drain = acc_empty + ACC;
   uint64_t* sf_full = drain + 1;                // [kSFSlots]: stage scale factors are in TMEM slot i
-  uint64_t* cp_drain = sf_full + C::kSFSlots;   // the copier's last copies have completed
+  uint64_t* cp_drain = sf_full + C::kSFSlots;   // the copier warps' last copies have completed
   // [S]: a stage's scale factors have landed.  With a separate copier they complete on
-  // their own barrier (and are issued first), so that the copier moves them into TMEM
+  // their own barrier (and are issued first), so that the copier warps move them into TMEM
   // while the stage's operand tiles are still arriving; otherwise they complete on full.
   uint64_t* sf_landed = cp_drain + 1;
   volatile int* s_abort = reinterpret_cast<volatile int*>(sf_landed + S);
@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
           const uint32_t sfa_t = tmem + sf_col0 + slot * C::kSFSlot;
           const uint32_t sfb_t = sfa_t + C::kSFACols;
           if constexpr (C::kSepCp) {
-            // the copier has put this stage's scale factors into the slot
+            // the copier warps have put this stage's scale factors into the slot
             if (!mbar_wait(&sf_full[slot], (nstage / C::kSFSlots) & 1, s_abort)) {
               latch_timeout(s_abort, p.status);
               ok = false;
