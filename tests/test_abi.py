@@ -94,6 +94,10 @@ def test_gemm_rejects_bad_arguments():
                               None, 0, None) == fp4.ERR_INVALID_ARG
     assert L.fp4_gemm_grouped(fp4.MXFP4, 4, 16, 16, 16, None, 16, 16, None, 64, 100, 64, 16, fp4.BF16,
                               None, 0, None) == fp4.ERR_INVALID_ARG   # N % 128
+    assert L.fp4_gemm_grouped(fp4.MXFP4, 1025, 16, 16, 16, None, 16, 16, None, 64, 128, 64, 16, fp4.BF16,
+                              None, 0, None) == fp4.ERR_INVALID_ARG   # more than 1024 groups
+    assert L.fp4_gemm_grouped(fp4.MXFP4, 4, None, 16, 16, None, 16, 16, None, 64, 128, 64, 16, fp4.BF16,
+                              None, 0, None) == fp4.ERR_INVALID_ARG   # no offsets
 
 
 def test_gemm_ex_rejects_unknown_flags():
