@@ -366,7 +366,7 @@ def _copies(per_copy_bytes: int) -> int:
 def _line(workload: str, value, unit: str, ms: float, args, extra: dict) -> dict:
     res = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "data": "synthetic (seeded, see DESIGN.md)", "config": {"workload": workload}}
+           "vs_baseline": None, "data": "synthetic (seeded, same recipes as the tests)", "config": {"workload": workload}}
     res.update(extra)
     return res
 

@@ -314,11 +314,11 @@ fp4_status fp4_gemm_bf16a(const void* X, const uint8_t* B, const uint8_t* sB, co
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------
-// Allocation-free GEMM.  Callers that cannot allocate device memory -- code running
-// while a CUDA graph is being captured, or a host (plugin runtime, embedded engine)
-// that owns every device byte and hands this library no allocator -- still need the
-// split-K scratch that decode-sized GEMMs use.  This variant takes it from a fixed
-// array compiled into the library instead of from the caller.
+// Allocation-free GEMM.  Some callers cannot allocate device memory: a host (plugin
+// runtime, embedded engine) that owns every device byte and hands this library no
+// allocator.  They still need the split-K scratch that decode-sized GEMMs use, so this
+// variant takes it from a fixed array compiled into the library instead of from the
+// caller.
 namespace fp4 {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB on every device that loads the library
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

@@ -182,16 +182,17 @@ fp4_status fp4_gemm_bf16a(const void* X_dev, const uint8_t* B_dev, const uint8_t
                           void* workspace_dev, size_t workspace_bytes, unsigned flags, void* stream);
 
 /* fp4_gemm for callers that cannot allocate device memory.  The pages have no
- * counterpart to this entry point: it exists for code that runs while a CUDA graph is
- * being captured (allocation is not allowed there) and for hosts -- plugin runtimes,
- * embedded engines -- that own all device memory and give this library no allocator.
+ * counterpart to this entry point.  Some hosts own every byte of device memory and give
+ * this library no allocator: plugin runtimes and embedded inference engines that carve
+ * one arena out of the GPU at start-up and treat any later cudaMalloc as a failure.
  * Arguments as fp4_gemm minus the workspace.  The split-K scratch that decode-sized
  * problems need comes from a fixed 4 MiB array compiled into the library, which every
  * GPU that loads the library holds until the process exits; shapes whose scratch
  * (fp4_gemm_workspace_size) exceeds 4 MiB return FP4_ERR_INVALID_ARG.  The first call
- * on a device looks up the array's device address (make it before any stream capture).
- * Every call clears the part of the array it uses, and all calls on a device share the
- * array: calls that overlap on the GPU race.  Allocates nothing. */
+ * on a device looks up the array's device address with cudaGetSymbolAddress, so make
+ * that first call before any stream capture.  Every call clears the part of the array
+ * it uses, and all calls on a device share the array: calls that overlap on the GPU
+ * race.  Calls no cudaMalloc or cudaFree. */
 fp4_status fp4_gemm_noalloc(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,
                             const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
                             int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,

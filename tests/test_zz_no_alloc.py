@@ -1,10 +1,13 @@
-"""fp4_gemm_noalloc: the GEMM entry point for callers that cannot allocate device memory
-(for example while a CUDA graph is being captured, or inside a host that owns all device
-memory and gives the library no allocator).  Its split-K scratch is a fixed array inside
-the library.  The test calls it twice in a row through the C ABI on a decode-shaped
-problem, which needs that scratch, and checks each result against fp4_gemm with a
-caller workspace, within the GEMM tolerance the other tests use.  It lives in its own
-file so that it runs after every other test."""
+"""fp4_gemm_noalloc: the GEMM entry point for callers that cannot allocate device memory,
+such as a host that owns all device memory and gives this library no allocator.  Its
+split-K scratch is a fixed array inside the library.
+
+The tests call it twice in a row through the C ABI:
+- a decode-shaped problem, which needs that scratch;
+- a tile-mode problem, which needs none.
+Each result is checked against the oracle's FP64 product at the GEMM tolerance the other
+tests use, and against fp4_gemm with a caller workspace at the same tolerance.  The file
+is named so that pytest collects it last."""
 import numpy as np
 import pytest
 import torch
@@ -16,26 +19,29 @@ from fp4_testutil import dequant_oracle, oracle_quantize, random_input
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_gemm_matches_workspace_gemm_twice():
-    m, n, k = 16, 3072, 4096
-    assert fp4.fp4_gemm_workspace_size(m, n, k, fp4.NVFP4) > 0   # this shape uses scratch
+@pytest.mark.parametrize("m,n,k", [(16, 3072, 4096),    # split over K: uses the built-in scratch
+                                   (512, 512, 512)])    # whole tiles: no scratch at all
+def test_noalloc_gemm_matches_oracle_and_workspace_gemm_twice(m, n, k):
+    need = fp4.fp4_gemm_workspace_size(m, n, k, fp4.NVFP4)
+    assert (need > 0) == (m == 16)
     xa = random_input(m, k, 91, torch.bfloat16)
     xb = random_input(n, k, 92, torch.float32, std=0.02, outliers=False)
     qa = fp4.quantize(xa.cuda(), fp4.NVFP4, 16)
     qb = fp4.quantize(xb.cuda(), fp4.NVFP4, 16)
-    ref = fp4.gemm(qa, qb, torch.float32)
-    torch.cuda.synchronize()
-    # tolerance base: sum_k |a_k b_k| over the oracle's dequantized operands
+    ref = fp4.gemm(qa, qb, torch.float32).cpu().numpy().astype(np.float64)
     oa, ob = oracle_quantize(xa, fp4.NVFP4, 16), oracle_quantize(xb, fp4.NVFP4, 16)
-    _, s = oracle.gemm_reference(dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4))
-    tol = oracle.gemm_tolerance(ref.cpu().numpy().astype(np.float64), s, bf16_out=False)
+    d_ref, s = oracle.gemm_reference(dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4))
+    tol = oracle.gemm_tolerance(d_ref, s, bf16_out=False)
+    assert np.all(np.abs(ref - d_ref) <= tol)
     for call in range(2):
         d = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
         fp4.fp4_gemm_noalloc(fp4.NVFP4, qa.codes, qa.scales, qa.g, qb.codes, qb.scales, qb.g, m, n, k, d, fp4.F32)
         torch.cuda.synchronize()
         assert fp4.fp4_get_status() == fp4.OK
-        err = np.abs(d.cpu().numpy().astype(np.float64) - ref.cpu().numpy().astype(np.float64))
-        assert np.all(err <= 2 * tol), f"call {call}: max err {err.max()}"
+        got = d.cpu().numpy().astype(np.float64)
+        err = np.abs(got - d_ref)
+        assert np.all(err <= tol), f"call {call}: max err / tol {np.max(err / tol)}"
+        assert np.all(np.abs(got - ref) <= tol), f"call {call}: differs from fp4_gemm"
 
 
 def test_noalloc_gemm_rejects_shapes_beyond_its_scratch():
