@@ -82,6 +82,8 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_e2m1_encode_sr": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_uint32]),
         "orc_rht16": (I32, [P, I64, I64, I32, ctypes.c_uint32, P]),
         "orc_quantize_mxfp4_1d": (I32, [P, I64, I64, I32, P, P]),
+        "orc_quantize_mxfp4_1d_r": (I32, [P, I64, I64, I32, I32, P, P]),
+        "orc_e8m0_encode_floor": (ctypes.c_uint8, [ctypes.c_float]),
         "orc_quantize_nvfp4_2d": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
         "orc_scales_bytes": (I64, [I64, I64]),
         "orc_swizzle_offset": (I64, [I64, I64, I64]),
@@ -175,13 +177,19 @@ def global_scale(amax_t: float) -> np.float32:
     return np.float32(_L().orc_global_scale(amax_t))
 
 
-def quantize(x: np.ndarray, fmt: int = NVFP4, block: int = 16, g_in=None):
+def e8m0_encode_floor(amax_b: float) -> int:
+    """E8M0 scale code rounded down: 2^(floor(log2 amax_b) - 2), by brute force."""
+    return int(_L().orc_e8m0_encode_floor(ctypes.c_float(amax_b)))
+
+
+def quantize(x: np.ndarray, fmt: int = NVFP4, block: int = 16, g_in=None, e8m0_floor: bool = False):
     """Quantize a row-major [rows, cols] tensor.
 
     Returns a dict with ``codes`` [rows, cols/2] uint8 (even element in the low
     nibble), ``scales`` row-major [rows, cols/16 or /32] uint8, ``g`` (float32; 1.0
     for MXFP4) and, for the 16x16 mode (block=256), ``codesT`` [cols, rows/2] and
-    ``scalesT`` [cols, rows/16].
+    ``scalesT`` [cols, rows/16].  ``e8m0_floor`` (MXFP4 only) picks the rounded-down
+    power-of-two scale instead of the nearest one.
     """
     x, dt = _as_input(x)
     if x.ndim == 1:
@@ -202,7 +210,7 @@ def quantize(x: np.ndarray, fmt: int = NVFP4, block: int = 16, g_in=None):
     elif fmt == MXFP4 and block == 32:
         codes = np.zeros((rows, cols // 2), np.uint8)
         sc = np.zeros((rows, cols // 32), np.uint8)
-        rc = L.orc_quantize_mxfp4_1d(_ptr(x), rows, cols, dt, _ptr(codes), _ptr(sc))
+        rc = L.orc_quantize_mxfp4_1d_r(_ptr(x), rows, cols, dt, 1 if e8m0_floor else 0, _ptr(codes), _ptr(sc))
         out.update(codes=codes, scales=sc, g=np.float32(1.0))
     elif fmt == NVFP4 and block == 256:
         codes = np.zeros((rows, cols // 2), np.uint8)
@@ -214,6 +222,8 @@ def quantize(x: np.ndarray, fmt: int = NVFP4, block: int = 16, g_in=None):
         out.update(codes=codes, scales=sc, codesT=codesT, scalesT=scT, g=np.float32(gbuf[0]))
     else:
         raise ValueError(f"unsupported fmt/block {fmt}/{block}")
+    if e8m0_floor and fmt != MXFP4:
+        raise ValueError("e8m0_floor applies to MXFP4 only")
     if rc != 0:
         raise NonFiniteInput("non-finite element")
     return out

@@ -286,9 +286,24 @@ static uint8_t nvfp4_encode_block(const float* xs, int n, float amax_b, float g,
     return sb;
 }
 
-/* One MXFP4 block of 32 values, E8M0 scale ([P2] MXFP4 passage; [P4]). */
-static uint8_t mxfp4_encode_block(const float* xs, int n, float amax_b, uint8_t* codes) {
-    uint8_t sb = orc_e8m0_encode(amax_b / 6.0f);
+/* The other way to reach a power of two ([P2] MXFP4 passage: a scale of 70 must become
+ * 64 or 128, so one may also round down): take the largest power of two not above the
+ * block amax and divide it by 4, the largest power of two on the E2M1 grid.  The block's
+ * largest element then lands in [4, 8) after scaling (values from 6 up saturate).  Brute
+ * force: the largest code c with 4 * 2^(c-127) <= amax_b; code 0 if none (and for a
+ * zero block). */
+uint8_t orc_e8m0_encode_floor(float amax_b) {
+    double a = (double)amax_b;
+    int best = 0;
+    for (int c = 0; c <= 254; ++c)
+        if (4.0 * e8m0_value(c) <= a) best = c;
+    return (uint8_t)best;
+}
+
+/* One MXFP4 block of 32 values, E8M0 scale ([P2] MXFP4 passage; [P4]): the nearest power
+ * of two of amax_b / 6, or (floor != 0) the rounded-down scale above. */
+static uint8_t mxfp4_encode_block(const float* xs, int n, float amax_b, int floor_mode, uint8_t* codes) {
+    uint8_t sb = floor_mode ? orc_e8m0_encode_floor(amax_b) : orc_e8m0_encode(amax_b / 6.0f);
     /* multiplying by 2^(127 - sb) is exact in FP32 (the factor is representable and
      * the scaling only moves the exponent), so it equals dividing by the scale */
     float f = (float)ldexp(1.0, 127 - (int)sb);
@@ -346,8 +361,18 @@ int orc_quantize_nvfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
     return orc_quantize_nvfp4_1d_r(x, rows, cols, dtype, g_in, NULL, codes, scales_rm, g_out);
 }
 
+int orc_quantize_mxfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype, int floor_mode,
+                            uint8_t* codes, uint8_t* scales_rm);
+
 int orc_quantize_mxfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
                           uint8_t* codes, uint8_t* scales_rm) {
+    return orc_quantize_mxfp4_1d_r(x, rows, cols, dtype, 0, codes, scales_rm);
+}
+
+/* floor_mode: 0 = nearest power of two of amax_b / 6; 1 = rounded down (see
+ * orc_e8m0_encode_floor). */
+int orc_quantize_mxfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype, int floor_mode,
+                            uint8_t* codes, uint8_t* scales_rm) {
     float xs[32];
     uint8_t cb[32];
     uint8_t* row_codes = (uint8_t*)malloc((size_t)cols);
@@ -359,7 +384,7 @@ int orc_quantize_mxfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
                 if (!isfinite(xs[i])) { free(row_codes); return ORC_ERR_NONFINITE; }
                 if (fabsf(xs[i]) > amax_b) amax_b = fabsf(xs[i]);
             }
-            scales_rm[r * (cols / 32) + b] = mxfp4_encode_block(xs, 32, amax_b, cb);
+            scales_rm[r * (cols / 32) + b] = mxfp4_encode_block(xs, 32, amax_b, floor_mode, cb);
             memcpy(row_codes + b * 32, cb, 32);
         }
         pack_row(row_codes, cols, codes + r * (cols / 2));

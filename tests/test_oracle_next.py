@@ -204,3 +204,63 @@ def test_epilogue_order_scale_bias_activation():
     assert np.array_equal(got, want)
     assert np.array_equal(oracle.epilogue(d), d)
     assert np.array_equal(oracle.epilogue(d, bias), d + bias[None, :])
+
+
+# ---------------------------------------------------------------- E8M0 rounded down
+# The MXFP4 scale may also be rounded down to a power of two ("MXFP4 / NVFP4 video
+# transcript", MXFP4 passage: 70 must become 64 or 128).  Reading: the largest power of two
+# not above the block amax, divided by 4 (the largest power of two on the E2M1 grid), so
+# that the block's largest element lands in [4, 8) after scaling.
+@pytest.mark.parametrize("amax,code", [
+    (6.0, 127), (4.0, 127), (3.99, 126), (8.0, 128), (7.99, 127), (0.75, 124), (1.0, 125),
+    (420.0, 133),            # scale 420 / 6 = 70 becomes 64 = 2^6, code 127 + 6
+    (0.0, 0), (2.0 ** -126, 0), (2.0 ** -124, 1), (2.0 ** 127, 252)])
+def test_e8m0_floor_hand_cases(amax, code):
+    assert oracle.e8m0_encode_floor(amax) == code
+
+
+def test_e8m0_floor_puts_the_block_amax_in_four_to_eight():
+    rng = np.random.default_rng(11)
+    for a in np.float32(2.0) ** rng.uniform(-100, 100, 2000).astype(np.float32):
+        x = oracle.e8m0_decode(oracle.e8m0_encode_floor(float(a)))
+        assert 4.0 * x <= float(a) < 8.0 * x, (a, x)
+
+
+def test_e8m0_floor_never_above_nearest():
+    """The rounded-down scale is within one binade of the nearest power of two of amax / 6
+    (both are powers of two within a factor of two of amax / 6 or of amax / 4, and
+    amax / 4 is 1.5 times amax / 6)."""
+    rng = np.random.default_rng(12)
+    for a in np.float32(2.0) ** rng.uniform(-60, 60, 2000).astype(np.float32):
+        f = oracle.e8m0_encode_floor(float(a))
+        n = int(oracle.e8m0_encode(np.array([np.float32(a) / np.float32(6.0)], np.float32))[0])
+        assert n - 1 <= f <= n + 1, (a, f, n)
+
+
+def test_quantize_mxfp4_floor_block_maximum_codes():
+    """With the rounded-down scale every non-zero block's largest element encodes as 4 or 6
+    (its scaled magnitude is in [4, 8): 4..5 rounds to 4, 5..8 to 6), and the codes equal
+    a plain E2M1 encode of x / scale."""
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((8, 256)) * np.float32(2.0) ** rng.integers(-20, 20, (8, 1))).astype(np.float32)
+    q = oracle.quantize(x, oracle.MXFP4, 32, e8m0_floor=True)
+    codes = np.zeros((8, 256), np.uint8)
+    codes[:, 0::2] = q["codes"] & 15
+    codes[:, 1::2] = q["codes"] >> 4
+    for r in range(8):
+        for b in range(8):
+            blk = x[r, b * 32:(b + 1) * 32]
+            sc = q["scales"][r, b]
+            assert sc == oracle.e8m0_encode_floor(float(np.abs(blk).max()))
+            scale = np.float32(oracle.e8m0_decode(sc))
+            want = oracle.e2m1_encode(blk / scale)      # exact: scale is a power of two
+            assert np.array_equal(codes[r, b * 32:(b + 1) * 32], want)
+            top = int(codes[r, b * 32 + int(np.abs(blk).argmax())] & 7)
+            assert GRID[top] in (4.0, 6.0)
+
+
+def test_quantize_mxfp4_floor_off_is_the_nearest_quantizer():
+    x = np.random.default_rng(14).standard_normal((4, 128)).astype(np.float32)
+    a = oracle.quantize(x, oracle.MXFP4, 32)
+    b = oracle.quantize(x, oracle.MXFP4, 32, e8m0_floor=False)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])

@@ -125,6 +125,18 @@ C_MUTATIONS = [
      "if ((signs >> i) & 1u) v[i] = -v[i];",
      "if ((signs >> (15 - i)) & 1u) v[i] = -v[i];",
      [lambda: tn.test_rht_spreads_a_spike_evenly(0x00FF, 0), tn.test_rht_fp32_within_the_butterfly_bound]),
+    ("E8M0 rounded down from amax / 6 instead of amax / 4",
+     "if (4.0 * e8m0_value(c) <= a) best = c;",
+     "if (6.0 * e8m0_value(c) <= a) best = c;",
+     [lambda: tn.test_e8m0_floor_hand_cases(4.0, 127), tn.test_e8m0_floor_puts_the_block_amax_in_four_to_eight]),
+    ("E8M0 rounded down one binade too far",
+     "if (4.0 * e8m0_value(c) <= a) best = c;",
+     "if (8.0 * e8m0_value(c) <= a) best = c;",
+     [lambda: tn.test_e8m0_floor_hand_cases(6.0, 127), tn.test_quantize_mxfp4_floor_block_maximum_codes]),
+    ("MXFP4 quantizer ignores the rounding mode",
+     "uint8_t sb = floor_mode ? orc_e8m0_encode_floor(amax_b) : orc_e8m0_encode(amax_b / 6.0f);",
+     "uint8_t sb = orc_e8m0_encode(amax_b / 6.0f);",
+     [tn.test_quantize_mxfp4_floor_block_maximum_codes]),
     ("Hadamard butterfly difference reversed",
      "v[j + h] = p - q;",
      "v[j + h] = q - p;",
