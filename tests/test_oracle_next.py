@@ -264,3 +264,30 @@ def test_quantize_mxfp4_floor_off_is_the_nearest_quantizer():
     a = oracle.quantize(x, oracle.MXFP4, 32)
     b = oracle.quantize(x, oracle.MXFP4, 32, e8m0_floor=False)
     assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])
+
+
+# ---------------------------------------------------------------- epilogue tolerance
+def test_epilogue_tolerance_covers_an_fp32_epilogue():
+    """An FP32 epilogue of an FP32-accurate product (the product rounded once, the bias
+    added in FP32, ReLU) stays inside the bound; the same bound without its bias term
+    does not cover large biases."""
+    rng = np.random.default_rng(21)
+    d = rng.standard_normal((64, 96)) * 3.0
+    s = np.abs(d) + 1.0
+    bias = (rng.standard_normal(96) * 1000.0).astype(np.float32).astype(np.float64)  # the bias is FP32 data
+    t_ref = oracle.epilogue(d, bias, "relu")
+    t32 = np.maximum(d.astype(np.float32) + bias.astype(np.float32), np.float32(0)).astype(np.float64)
+    tol = oracle.epilogue_tolerance(t_ref, d, s, bias, False)
+    assert np.all(np.abs(t32 - t_ref) <= tol)
+    no_bias_term = 1e-6 * s + 2.0 ** -24 * np.abs(d)
+    assert np.any(np.abs(t32 - t_ref) > no_bias_term)
+
+
+def test_epilogue_tolerance_reduces_to_the_gemm_tolerance_without_bias():
+    rng = np.random.default_rng(22)
+    d = rng.standard_normal((8, 16))
+    s = np.abs(d) + 0.5
+    tol = oracle.epilogue_tolerance(d, d, s, None, True)
+    base = oracle.gemm_tolerance(d, s, True)
+    # the extra FP32 rounding term is the only difference
+    assert np.all(tol >= base) and np.all(tol - base <= 2.0 ** -24 * (np.abs(d) + 1e-6 * s) * (1 + 1e-9) + 1e-300 + 0.5 * oracle.bf16_ulp(np.abs(d) + tol))
