@@ -26,6 +26,8 @@ NVFP4, MXFP4 = 0, 1
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = range(6)
 GEMM_WEIGHTS_READY = 1
+QUANT_E8M0_FLOOR = 1
+ACT_NONE, ACT_RELU = 0, 1
 _STATUS_NAMES = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED", 3: "FP4_ERR_CUDA",
                  4: "FP4_ERR_TIMEOUT", 5: "FP4_ERR_NONFINITE"}
 
@@ -58,11 +60,18 @@ def lib() -> ctypes.CDLL:
                 "fp4_amax": (I32, [P, I64, I32, P, P, SZ, P]),
                 "fp4_quantize": (I32, [P, I64, I64, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]),
                 "fp4_quantize_grouped": (I32, [P, I64, I64, I32, I32, I32, P, P, P, P, P, P, SZ, P]),
+                "fp4_quantize_ex": (I32, [P, I64, I64, I32, I32, I32, ctypes.c_uint, P, P, P, P, P, P, P, SZ, P]),
+                "fp4_quantize_sr": (I32, [P, I64, I64, I32, P, P, P, P, P, P, SZ, P]),
+                "fp4_quantize_rht": (I32, [P, I64, I64, I32, I32, ctypes.c_uint32, P, P, P, P, P, SZ, P]),
+                "fp4_global_scale": (I32, [P, P, P]),
                 "fp4_dequantize": (I32, [P, P, P, I64, I64, I32, P, P]),
                 "fp4_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
                 "fp4_gemm": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_gemm_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_noalloc": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
+                "fp4_gemm_epilogue_workspace_size": (SZ, [I64, I64, I64, I32, I32]),
+                "fp4_gemm_epilogue": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, I32, P, P, P, P, SZ,
+                                            P]),
                 "fp4_gemm_bf16a_workspace_size": (SZ, [I64, I64, I64]),
                 "fp4_gemm_bf16a": (I32, [P, P, P, P, I64, I64, I64, P, I32, P, P, P, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_grouped": (I32, [I32, I32, P, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
@@ -150,6 +159,30 @@ def fp4_quantize_grouped(x, rows, cols, in_dtype, fmt, num_groups, offsets, code
                                       workspace_bytes, _s(stream)))
 
 
+def fp4_quantize_ex(x, rows, cols, in_dtype, fmt, block, flags, codes_out, scales_out, global_out,
+                    codesT_out=None, scalesT_out=None, global_in=None, workspace=None, workspace_bytes=0,
+                    stream=None):
+    _check(lib().fp4_quantize_ex(_p(x), rows, cols, in_dtype, fmt, block, flags, _p(codes_out), _p(scales_out),
+                                 _p(global_out), _p(codesT_out), _p(scalesT_out), _p(global_in), _p(workspace),
+                                 workspace_bytes, _s(stream)))
+
+
+def fp4_quantize_sr(x, rows, cols, in_dtype, rbits, codes_out, scales_out, global_out, global_in=None,
+                    workspace=None, workspace_bytes=0, stream=None):
+    _check(lib().fp4_quantize_sr(_p(x), rows, cols, in_dtype, _p(rbits), _p(codes_out), _p(scales_out),
+                                 _p(global_out), _p(global_in), _p(workspace), workspace_bytes, _s(stream)))
+
+
+def fp4_quantize_rht(x, rows, cols, in_dtype, fmt, signs, codes_out, scales_out, global_out, global_in=None,
+                     workspace=None, workspace_bytes=0, stream=None):
+    _check(lib().fp4_quantize_rht(_p(x), rows, cols, in_dtype, fmt, signs, _p(codes_out), _p(scales_out),
+                                  _p(global_out), _p(global_in), _p(workspace), workspace_bytes, _s(stream)))
+
+
+def fp4_global_scale(amax, global_out, stream=None):
+    _check(lib().fp4_global_scale(_p(amax), _p(global_out), _s(stream)))
+
+
 def fp4_dequantize(codes, scales, global_, rows, cols, fmt, out, stream=None):
     _check(lib().fp4_dequantize(_p(codes), _p(scales), _p(global_), rows, cols, fmt, _p(out), _s(stream)))
 
@@ -163,6 +196,17 @@ def fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace=None
                 stream=None):
     _check(lib().fp4_gemm_ex(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(D), out_dtype,
                              _p(workspace), workspace_bytes, flags, _s(stream)))
+
+
+def fp4_gemm_epilogue_workspace_size(M: int, N: int, K: int, fmt: int, fp4_out: bool) -> int:
+    return int(lib().fp4_gemm_epilogue_workspace_size(M, N, K, fmt, 1 if fp4_out else 0))
+
+
+def fp4_gemm_epilogue(fmt, A, sA, gA, B, sB, gB, M, N, K, bias, act, D, out_dtype, Dcodes=None, Dscales=None,
+                      gD=None, workspace=None, workspace_bytes=0, stream=None):
+    _check(lib().fp4_gemm_epilogue(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(bias), act, _p(D),
+                                   out_dtype, _p(Dcodes), _p(Dscales), _p(gD), _p(workspace), workspace_bytes,
+                                   _s(stream)))
 
 
 def fp4_gemm_bf16a_workspace_size(M: int, N: int, K: int) -> int:

@@ -112,7 +112,8 @@ fp4_status fp4_amax(const void* x, int64_t n, fp4_dtype in_dtype, float* amax_ou
 static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
                                   int block, uint8_t* codes, uint8_t* scales, float* gout, uint8_t* codesT,
                                   uint8_t* scalesT, const float* gin, void* ws, size_t ws_bytes, int num_groups,
-                                  const int32_t* offsets, void* stream) {
+                                  const int32_t* offsets, void* stream, int variant = kQuantPlain,
+                                  const uint32_t* rbits = nullptr, uint32_t signs = 0) {
   if (!x || !codes || !scales) return fail(FP4_ERR_INVALID_ARG, "null pointer");
   if (rows <= 0 || cols <= 0) return fail(FP4_ERR_INVALID_ARG, "rows and cols must be positive");
   if (cols % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "cols must be a multiple of 32");
@@ -130,6 +131,10 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
       (scalesT && !aligned16(scalesT)))
     return fail(FP4_ERR_INVALID_ARG, "x, codes and scales must be 16-byte aligned");
   if (num_groups && (num_groups > kMaxGroups || !offsets)) return fail(FP4_ERR_INVALID_ARG, "groups / offsets");
+  if (variant != kQuantPlain && two_d) return fail(FP4_ERR_UNSUPPORTED, "quantizer variants are 1-D only");
+  if (variant == kQuantMxFloor && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "the E8M0 floor is for MXFP4");
+  if (variant == kQuantSR && (fmt != FP4_NVFP4 || !rbits || !aligned16(rbits)))
+    return fail(FP4_ERR_INVALID_ARG, "stochastic rounding: NVFP4, 16-byte aligned random words");
   const bool need_amax = fmt == FP4_NVFP4 && !gin;
   if (need_amax && (!ws || ws_bytes < kQuantWorkspaceBytes || !aligned16(ws)))
     return fail(FP4_ERR_INVALID_ARG, "workspace too small or misaligned (fp4_quantize_workspace_size)");
@@ -140,7 +145,7 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   const int bf16 = in_dtype == FP4_BF16;
   const int mx = fmt == FP4_MXFP4;
   cudaError_t e = cudaSuccess;
-  if (!two_d && !num_groups && quantize_small_fits(rows, cols, bf16, mx)) {
+  if (variant == kQuantPlain && !two_d && !num_groups && quantize_small_fits(rows, cols, bf16, mx)) {
     // one launch: amax, global scale and encode by one thread-block cluster
     e = launch_quantize_small(x, rows, cols, bf16, mx, codes, scales, mx ? nullptr : gin, gout, status, st);
     return e == cudaSuccess ? FP4_OK : cuda_fail(e, "quantize launch");
@@ -148,7 +153,8 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   const float* g = nullptr;
   if (fmt == FP4_NVFP4) {
     if (need_amax) {
-      e = launch_amax(x, rows * cols, bf16, static_cast<uint32_t*>(ws), nullptr, gout, status, st);
+      e = launch_amax(x, rows * cols, bf16, static_cast<uint32_t*>(ws), nullptr, gout, status, st,
+                      variant == kQuantRHT, signs);
       if (e != cudaSuccess) return cuda_fail(e, "amax launch");
       g = gout;
     } else {
@@ -165,7 +171,8 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   if (two_d)
     e = launch_quantize_2d(x, rows, cols, bf16, codes, scales, codesT, scalesT, g, status, st);
   else
-    e = launch_quantize_1d(x, rows, cols, bf16, mx, codes, scales, g, offsets, num_groups, status, st);
+    e = launch_quantize_1d(x, rows, cols, bf16, mx, codes, scales, g, offsets, num_groups, status, st, variant, rbits,
+                           signs);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "quantize launch");
 }
 
@@ -175,6 +182,41 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, fp4_dtype in_
                         void* stream) {
   return quantize_common(x, rows, cols, in_dtype, fmt, block, codes_out, scales_out, global_out, codesT_out,
                          scalesT_out, global_in, workspace, workspace_bytes, 0, nullptr, stream);
+}
+
+fp4_status fp4_quantize_ex(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt, int block,
+                           unsigned flags, uint8_t* codes_out, uint8_t* scales_out, float* global_out,
+                           uint8_t* codesT_out, uint8_t* scalesT_out, const float* global_in, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(FP4_QUANT_E8M0_FLOOR)) return fail(FP4_ERR_INVALID_ARG, "unknown flag");
+  return quantize_common(x, rows, cols, in_dtype, fmt, block, codes_out, scales_out, global_out, codesT_out,
+                         scalesT_out, global_in, workspace, workspace_bytes, 0, nullptr, stream,
+                         (flags & FP4_QUANT_E8M0_FLOOR) ? kQuantMxFloor : kQuantPlain);
+}
+
+fp4_status fp4_quantize_sr(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, const uint32_t* rbits,
+                           uint8_t* codes_out, uint8_t* scales_out, float* global_out, const float* global_in,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return quantize_common(x, rows, cols, in_dtype, FP4_NVFP4, 16, codes_out, scales_out, global_out, nullptr, nullptr,
+                         global_in, workspace, workspace_bytes, 0, nullptr, stream, kQuantSR, rbits, 0);
+}
+
+fp4_status fp4_quantize_rht(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
+                            uint32_t signs, uint8_t* codes_out, uint8_t* scales_out, float* global_out,
+                            const float* global_in, void* workspace, size_t workspace_bytes, void* stream) {
+  if (signs > 0xFFFFu) return fail(FP4_ERR_INVALID_ARG, "signs: 16 bits");
+  return quantize_common(x, rows, cols, in_dtype, fmt, fmt == FP4_MXFP4 ? 32 : 16, codes_out, scales_out, global_out,
+                         nullptr, nullptr, global_in, workspace, workspace_bytes, 0, nullptr, stream, kQuantRHT,
+                         nullptr, signs);
+}
+
+fp4_status fp4_global_scale(const float* amax, float* global_out, void* stream) {
+  if (!amax || !global_out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  const cudaError_t e = launch_global_scale(amax, global_out, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "global scale launch");
 }
 
 fp4_status fp4_quantize_grouped(const void* x, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
@@ -208,11 +250,11 @@ size_t fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt) {
 static fp4_status gemm_common(const GemmProblem& g, fp4_fmt fmt, fp4_dtype out_dtype, void* stream) {
   if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "fmt");
   if (out_dtype != FP4_F32 && out_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "out_dtype");
-  if (!g.A || !g.B || !g.sA || !g.sB || !g.D) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!g.A || !g.B || !g.sA || !g.sB || (!g.D && !g.q_codes)) return fail(FP4_ERR_INVALID_ARG, "null pointer");
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(FP4_ERR_INVALID_ARG, "M, N, K must be positive");
   if (g.K % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "K must be a multiple of 32");
   if (g.M > (1ll << 31) - 256 || g.N > (1ll << 31) - 256) return fail(FP4_ERR_UNSUPPORTED, "dimension too large");
-  if (!aligned16(g.A) || !aligned16(g.B) || !aligned16(g.sA) || !aligned16(g.sB) || !aligned16(g.D))
+  if (!aligned16(g.A) || !aligned16(g.B) || !aligned16(g.sA) || !aligned16(g.sB) || (g.D && !aligned16(g.D)))
     return fail(FP4_ERR_INVALID_ARG, "A, B, scales and D must be 16-byte aligned");
   unsigned* status;
   fp4_status s = device_state(&status);
@@ -253,6 +295,44 @@ fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const floa
                     const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, void* D, fp4_dtype out_dtype,
                     void* workspace, size_t workspace_bytes, void* stream) {
   return fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace, workspace_bytes, 0u, stream);
+}
+
+fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
+                             const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, const float* bias,
+                             fp4_act act, void* D, fp4_dtype out_dtype, uint8_t* Dcodes, uint8_t* Dscales,
+                             const float* gD, void* workspace, size_t workspace_bytes, void* stream) {
+  if (act != FP4_ACT_NONE && act != FP4_ACT_RELU) return fail(FP4_ERR_INVALID_ARG, "act");
+  if (!D && !Dcodes) return fail(FP4_ERR_INVALID_ARG, "no output: D and Dcodes are both NULL");
+  if (Dcodes && (!Dscales || !gD)) return fail(FP4_ERR_INVALID_ARG, "FP4 output needs Dscales and gD");
+  if (Dcodes && N % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "FP4 output needs N % 32 == 0");
+  if (Dcodes && (!aligned16(Dcodes) || !aligned16(Dscales))) return fail(FP4_ERR_INVALID_ARG, "Dcodes / Dscales alignment");
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return fail(FP4_ERR_INVALID_ARG, "bias alignment");
+  GemmProblem g{};
+  g.mx = fmt == FP4_MXFP4;
+  g.A = A;
+  g.sA = sA;
+  g.gA = gA;
+  g.B = B;
+  g.sB = sB;
+  g.gB = gB;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.D = D;
+  g.out_bf16 = out_dtype == FP4_BF16;
+  g.ws = workspace;
+  g.ws_bytes = workspace_bytes;
+  g.bias = bias;
+  g.act = act == FP4_ACT_RELU ? 1 : 0;
+  g.q_codes = Dcodes;
+  g.q_scales = Dscales;
+  g.q_g = gD;
+  return gemm_common(g, fmt, out_dtype, stream);
+}
+
+size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int fp4_out) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return gemm_workspace_bytes(M, N, K, fmt == FP4_MXFP4, fp4_out != 0);
 }
 
 size_t fp4_gemm_bf16a_workspace_size(int64_t M, int64_t N, int64_t K) {

@@ -54,6 +54,8 @@ struct DecodeArgs {
   int weights_ready;      // W was not written by the kernel just before this one
   unsigned* gbar;         // fused: [0] call counter, then one 128-byte slot per CTA
   unsigned* status;
+  const float* bias;      // [N] added to every output row after the scale, or null
+  int act;                // 0: none, 1: ReLU
 };
 
 // K steps of one segment at most (the activations' scale factors for a segment take 16
@@ -707,9 +709,16 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
             for (int j = 0; j < BN; ++j)
               if (j < p.M) __stcg(wsrow + j, 0.0f);
           }
+          // the epilogue after the scale: bias of this output column, then the activation
+          const float bias = p.bias ? __ldg(p.bias + row) : 0.0f;
 #pragma unroll
           for (int j = 0; j < BN; ++j)
-            if (j < p.M) d_store(p, row, j, v[j] * scale);
+            if (j < p.M) {
+              float o = v[j] * scale;
+              if (p.bias) o = __fadd_rn(o, bias);
+              if (p.act == 1) o = fmaxf(o, 0.0f);
+              d_store(p, row, j, o);
+            }
         }
         if (et == 0) p.tile_cnt[t] = 0;
         next_owned += np;
@@ -889,6 +898,8 @@ int launch_decode(const DecodeProblem& q, unsigned* status, cudaStream_t st, con
   a.gbar = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(q.ws) + ws_partials(q.M, q.N) + ws_counters(q.N));
   a.weights_ready = q.weights_ready;
   a.status = status;
+  a.bias = q.bias;
+  a.act = q.act;
   const int grid = pl.nseg * pl.ctas_per_seg;
   cudaError_t e;
   if (q.X) e = BN == 16 ? run_decode<16, true>(tw, tx, a, grid, st) : run_decode<32, true>(tw, tx, a, grid, st);

@@ -83,6 +83,14 @@ struct GemmArgs {
   const int32_t* offsets;
   int b_rows_per_group;
   unsigned* status;
+  // epilogue after the scale ("Rubin FP4 GEMM overview" 3.2 / 4.2): + bias[n], activation,
+  // and optionally an NVFP4 copy of the result (16-blocks along n, caller's global scale)
+  const float* bias;   // [N] (output columns), or null
+  int act;             // 0: none, 1: ReLU
+  uint8_t* q_codes;    // [M, N/2] NVFP4 codes of the result, or null
+  uint8_t* q_scales;   // swizzled scale atoms of the [M, N/16] block scales
+  const float* q_g;    // global scale of the NVFP4 result (device)
+  int64_t q_atoms;     // scale atoms per 128-row block of the result: ceil(N/16, 4) / 4
 };
 
 struct Work {
@@ -324,6 +332,58 @@ __device__ __forceinline__ void store_row16(const GemmArgs& p, int row, int col,
 #pragma unroll
   for (int j = 0; j < 16; ++j)
     if (col + j < p.Nk) store_out(p, base + j, v[j]);
+}
+
+// Bias and activation of 16 consecutive kernel columns [col, col+16) of kernel row `row`
+// (values already multiplied by gA * gB).  With swapped operands the kernel row is the
+// output column, which indexes the bias.
+__device__ __forceinline__ void epi_bias_act(const GemmArgs& p, int row, int col, float (&v)[16]) {
+  if (p.bias) {
+    if (p.transposed) {
+      const float b = p.bias[row];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], b);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (col + j < p.Nk) v[j] = __fadd_rn(v[j], __ldg(p.bias + col + j));
+    }
+  }
+  if (p.act == 1) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = fmaxf(v[j], 0.0f);
+  }
+}
+
+// NVFP4 copy of 16 output columns [col, col+16) of output row `row` (one block; the
+// caller guarantees N % 32 == 0 and a row-major kernel orientation): block scale and
+// codes exactly as the quantize kernels compute them, with the caller's global scale.
+__device__ __forceinline__ void epi_quantize16(const GemmArgs& p, int row, int col, const float (&v)[16]) {
+  const float g = *p.q_g;
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) m = max(m, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+  uint32_t sb;
+  const float mul = nvfp4_block_scale(__uint_as_float(m), g, sb);
+  float a[8], b[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    a[j] = v[j] == 0.0f ? v[j] : __fmul_rn(v[j], mul);  // a zero stays zero if 1/denom overflowed
+    b[j] = v[8 + j] == 0.0f ? v[8 + j] : __fmul_rn(v[8 + j], mul);
+  }
+  *reinterpret_cast<uint2*>(p.q_codes + static_cast<int64_t>(row) * (p.Nk / 2) + col / 2) =
+      make_uint2(pack8<kE2M1Hardware>(a), pack8<kE2M1Hardware>(b));
+  const int c = col / 16;
+  p.q_scales[((row / 128) * p.q_atoms + c / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4 + c % 4] =
+      static_cast<uint8_t>(sb);
+}
+
+// Finishes 16 consecutive kernel columns of one kernel row: bias, activation, the
+// BF16 / FP32 store and the NVFP4 copy.
+__device__ __forceinline__ void epi_row16(const GemmArgs& p, int row, int col, float (&v)[16]) {
+  epi_bias_act(p, row, col, v);
+  if (p.out) store_row16(p, row, col, v);
+  if (p.q_codes && col < p.Nk) epi_quantize16(p, row, col, v);
 }
 
 // Named barrier among the epilogue threads of one pipeline.
@@ -755,7 +815,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
     // BF16 row-major tiles whose columns are all in range are converted into registers
     // and TMEM is handed back to the MMA thread before the stores, so that they overlap
     // the next tile's MMAs
-    const bool early_release = C::kSepCp && p.mode != kModeStreamK && p.out_bf16 && !p.transposed && p.vec_store;
+    const bool early_release = C::kSepCp && p.mode != kModeStreamK && p.out && p.out_bf16 && !p.transposed &&
+                               p.vec_store && !p.q_codes;
     // hands an accumulator back to the MMA thread (a pair's leader counts both CTAs' warps)
     auto release_acc = [&](int a) {
       if constexpr (PAIR)
@@ -793,9 +854,12 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
           uint32_t rr[16];
           tmem_ld16(taddr + c0 + cw, rr);
           tmem_ld_wait();
+          float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 2)
-            pk[(cw + j) / 2] = pack_bf16x2(__uint_as_float(rr[j]) * scale, __uint_as_float(rr[j + 1]) * scale);
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]) * scale;
+          if (p.bias || p.act) epi_bias_act(p, row, w.n0 + c0 + cw, v);
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) pk[(cw + j) / 2] = pack_bf16x2(v[j], v[j + 1]);
         }
         tc_fence_before();
         __syncwarp();
@@ -837,7 +901,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]) * scale;
-            store_row16(p, row, col, v);
+            epi_row16(p, row, col, v);
           }
         }
         }
@@ -889,7 +953,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
                   }
                 }
               }
-              store_row16(p, row, col, v);
+              epi_row16(p, row, col, v);
             }
           }
           if (et == 0) p.tile_cnt[w.tile] = 0;
@@ -1035,7 +1099,7 @@ struct Plan {
   size_t ws_bytes;
 };
 
-static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
+static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx, bool row_major_out = false) {
   Plan pl{};
   pl.num_kb = static_cast<int>((K + 255) / 256);
   (void)mx;
@@ -1054,7 +1118,7 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
     pl.ws_bytes = 0;
     return pl;
   }
-  if (M <= 64) {  // decode: weight rows fill MMA-M, the few activation rows are MMA-N
+  if (M <= 64 && !row_major_out) {  // decode: weight rows fill MMA-M, the few activation rows are MMA-N
     pl.swap = true;
     pl.Mk = N;
     pl.Nk = M;
@@ -1095,9 +1159,9 @@ static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx) {
   return pl;
 }
 
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx) {
-  if (!mx && decode_eligible(M, N, K)) return decode_workspace_bytes(M, N);
-  return make_plan(M, N, K, 0, mx).ws_bytes;
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx, bool fp4_out) {
+  if (!mx && !fp4_out && decode_eligible(M, N, K)) return decode_workspace_bytes(M, N);
+  return make_plan(M, N, K, 0, mx, fp4_out).ws_bytes;
 }
 
 // the quantize workspace (tensor amax), then the GEMM's
@@ -1176,7 +1240,7 @@ static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtenso
 
 int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err) {
   const int grouped = g.num_groups > 0;
-  if (!grouped && !g.mx && decode_eligible(g.M, g.N, g.K)) {
+  if (!grouped && !g.mx && !g.q_codes && decode_eligible(g.M, g.N, g.K)) {
     // a few activation rows: the decode kernel (the weights are problem B)
     DecodeProblem q{};
     q.W = g.B;
@@ -1193,9 +1257,12 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
     q.ws = g.ws;
     q.ws_bytes = g.ws_bytes;
     q.weights_ready = g.weights_ready;
+    q.bias = g.bias;
+    q.act = g.act;
     return launch_decode(q, status, st, why, err);
   }
-  const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx);
+  // the NVFP4 copy of the result is written by rows: keep the operands in place
+  const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx, g.q_codes != nullptr);
   if (g.ws_bytes < pl.ws_bytes || (pl.ws_bytes && !g.ws)) {
     *why = "workspace too small (see fp4_gemm_workspace_size)";
     return 1;
@@ -1258,6 +1325,12 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   a.group_m = 16;
   a.total_units = pl.units;
   a.status = status;
+  a.bias = g.bias;
+  a.act = g.act;
+  a.q_codes = g.q_codes;
+  a.q_scales = g.q_scales;
+  a.q_g = g.q_g;
+  a.q_atoms = (g.N / 16 + 3) / 4;
   if (pl.mode == kModeStreamK) {
     a.ws = static_cast<float*>(g.ws);
     a.tile_cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(g.ws) + (static_cast<size_t>(g.M * g.N) * 4 + 255) / 256 * 256);

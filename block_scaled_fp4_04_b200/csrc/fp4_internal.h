@@ -22,11 +22,15 @@ constexpr bool kE2M1Hardware = FP4_E2M1_HW != 0;
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// rht != 0: the maximum of the 16-point Hadamard transform (sign bits `signs`) of x.
 cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float* amax_out, float* g_out,
-                        unsigned* status, cudaStream_t st);
+                        unsigned* status, cudaStream_t st, int rht = 0, uint32_t signs = 0);
+// Quantizer variants of the 1-D kernel (see fp4_quantize.cu).
+enum { kQuantPlain = 0, kQuantMxFloor = 1, kQuantSR = 2, kQuantRHT = 3 };
 cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
                                uint8_t* scales, const float* g, const int32_t* offsets, int num_groups,
-                               unsigned* status, cudaStream_t st);
+                               unsigned* status, cudaStream_t st, int variant = kQuantPlain,
+                               const uint32_t* rbits = nullptr, uint32_t signs = 0);
 // Small tensors (see quantize_small_fits): amax, global scale and 1-D quantize in one
 // launch of one thread-block cluster; the scale buffer is zero-filled and written.
 constexpr int kSmallCtas = 8, kSmallThreads = 512;
@@ -40,6 +44,8 @@ cudaError_t launch_quantize_2d(const void* x, int64_t rows, int64_t cols, int bf
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
                               int64_t cols, int mx, float* out, cudaStream_t st);
 cudaError_t launch_set_value(float* p, float v, cudaStream_t st);
+// g = amax / (6 * 448), 1 when amax is 0; a non-finite amax latches kStatusNonFinite.
+cudaError_t launch_global_scale(const float* amax, float* g, unsigned* status, cudaStream_t st);
 cudaError_t launch_debug_encode(const float* in, int64_t n, int which, uint8_t* out, cudaStream_t st);
 
 // GEMM problem as the host API sees it (see fp4.h for the meaning of each field).
@@ -56,9 +62,15 @@ struct GemmProblem {
   // grouped
   int num_groups;            // 0: plain GEMM
   const int32_t* offsets;
+  // epilogue after the scale: bias [N], activation (0 none, 1 ReLU), and an NVFP4 copy
+  // of the result (codes [M, N/2], swizzled scales of [M, N/16], caller's global scale)
+  const float* bias;
+  int act;
+  uint8_t *q_codes, *q_scales;
+  const float* q_g;
 };
 
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx);
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx, bool fp4_out = false);
 
 size_t gemm_bf16a_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -83,6 +95,8 @@ struct DecodeProblem {
   void* ws;
   size_t ws_bytes;
   int weights_ready;
+  const float* bias;  // [N] or null
+  int act;            // 0 none, 1 ReLU
 };
 bool decode_eligible(int64_t M, int64_t N, int64_t K);
 size_t decode_workspace_bytes(int64_t M, int64_t N);

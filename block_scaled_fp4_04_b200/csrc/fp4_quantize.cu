@@ -59,6 +59,75 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 
 __device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
+// ------------------------------------------------------------------ quantizer variants
+// Variants of the 1-D quantizer (the steps around the hot path, "MXFP4 / NVFP4 video
+// transcript", training-recipe and MXFP4 passages):
+//   kQuantPlain    the method as stated;
+//   kQuantMxFloor  MXFP4 with the block scale rounded down to a power of two;
+//   kQuantSR       NVFP4 with stochastic rounding of the elements (caller's random words);
+//   kQuantRHT      a 16-point random Hadamard transform of every 16-element block first.
+
+// Hadamard transform of the 16-element blocks that lanes hold EPC elements of: this
+// lane holds elements [j0, j0 + EPC) of its block (j0 = (lane % (16 / EPC)) * EPC), its
+// partners hold the rest.  Signs first (bit j of `signs` negates element j), then the
+// butterfly stages of half-width 1, 2, 4, 8 in that order (pair (j, j + h) becomes
+// (sum, difference)), then the exact factor 1/4: the same FP32 operations, in the same
+// order, as the definition.  Stages narrower than EPC stay in the thread; wider ones pair
+// lanes by a shuffle.  All lanes of the warp take part.
+template <int EPC>
+__device__ __forceinline__ void rht16_lanes(float (&v)[EPC], uint32_t signs, int j0) {
+#pragma unroll
+  for (int i = 0; i < EPC; ++i)
+    if ((signs >> (j0 + i)) & 1u) v[i] = -v[i];
+#pragma unroll
+  for (int h = 1; h < EPC; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < EPC; ++i)
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+#pragma unroll
+  for (int h = EPC; h < 16; h <<= 1) {
+    const int lane_bit = h / EPC;
+    const bool upper = ((j0 / EPC) & lane_bit) != 0;  // this lane holds the j + h half
+#pragma unroll
+    for (int i = 0; i < EPC; ++i) {
+      const float o = __shfl_xor_sync(0xFFFFFFFFu, v[i], lane_bit);
+      v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < EPC; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+}
+
+// Stochastic E2M1 rounding of a scaled value s with one 32-bit random word: |s| between
+// grid neighbours lo < |s| < hi goes up iff u < (|s| - lo) / (hi - lo), u = (bits >> 8)
+// * 2^-24.  The difference is exact (lo <= |s| < 2 lo, or lo = 0) and the gap a power of
+// two, so the fraction is exact in FP32.  Grid values stay, |s| >= 6 saturates; the sign
+// bit copies s's sign.
+__device__ __forceinline__ uint32_t e2m1_code_sr(float s, uint32_t bits) {
+  const float a = fabsf(s);
+  const uint32_t sign = (__float_as_uint(s) >> 28) & 8u;
+  if (a >= 6.0f) return 7u | sign;
+  const uint32_t lo = (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) + (a >= 4.0f);
+  const float lov = e2m1_value(lo);
+  if (a == lov) return lo | sign;
+  const float inv_gap = lo < 4 ? 2.0f : lo < 6 ? 1.0f : 0.5f;
+  const float frac = __fmul_rn(__fsub_rn(a, lov), inv_gap);
+  const float u = __fmul_rn(__uint2float_rn(bits >> 8), 5.9604644775390625e-08f);  // 2^-24
+  return (u < frac ? lo + 1u : lo) | sign;
+}
+
+// E8M0 scale rounded down: 2^(floor(log2 amax_b) - 2), i.e. the exponent field less 2,
+// clamped to [0, 254] (subnormal and zero amax give 0).
+__device__ __forceinline__ uint32_t e8m0_floor_code(float amax_b) {
+  const uint32_t e = __float_as_uint(amax_b) >> 23;
+  if (e >= 255u) return 254u;
+  return e >= 2u ? e - 2u : 0u;
+}
+
 // Programmatic dependent launch: let the next kernel on the stream start its prologue
 // early / wait until the previous kernel's writes are visible (no-ops without the
 // launch attribute).
@@ -70,17 +139,36 @@ __device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontro
 // the numeric order, and inf / NaN patterns exceed every finite one).  Each block writes
 // its partial; the last block to finish (ticket from a self-resetting atomicInc) reduces
 // them, latches non-finite input, and writes amax and / or g.
-template <typename T>
+// RHT: the maximum of the Hadamard-transformed values (n a multiple of 16; each thread
+// transforms whole 16-element blocks, in the same FP32 order as the quantize kernel).
+template <typename T, bool RHT = false>
 __global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, int64_t n, uint32_t* ws,
-                                                    float* amax_out, float* g_out, unsigned* status) {
+                                                    float* amax_out, float* g_out, unsigned* status,
+                                                    uint32_t signs) {
   allow_dependents();
   wait_prior_grids();  // x may be the output of the kernel just before
   constexpr int EPC = Elem<T>::kPerChunk;
-  const int64_t nchunks = n / EPC;
+  const int64_t nchunks = RHT ? 0 : n / EPC;
   const uint4* xc = reinterpret_cast<const uint4*>(x);
   uint32_t m = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if constexpr (RHT) {
+    constexpr int CPB = 16 / EPC;  // 16-byte chunks per 16-element block
+    for (int64_t b = i; b < n / 16; b += stride) {
+      float v[16];
+#pragma unroll
+      for (int c = 0; c < CPB; ++c) {
+        float t[EPC];
+        Elem<T>::unpack(ld_stream(xc + b * CPB + c), t);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) v[c * EPC + e] = t[e];
+      }
+      rht16_lanes<16>(v, signs, 0);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) m = max(m, abs_bits(v[e]));
+    }
+  }
   for (; i + 3 * stride < nchunks; i += 4 * stride) {
     uint4 u[4];
 #pragma unroll
@@ -99,7 +187,7 @@ __global__ void __launch_bounds__(512) amax_kernel(const T* __restrict__ x, int6
 #pragma unroll
     for (int e = 0; e < EPC; ++e) m = max(m, abs_bits(v[e]));
   }
-  if (blockIdx.x == 0) {  // tail elements that do not fill a 16-byte chunk
+  if (!RHT && blockIdx.x == 0) {  // tail elements that do not fill a 16-byte chunk
     for (int64_t t = nchunks * EPC + threadIdx.x; t < n; t += blockDim.x) {
       float v;
       if constexpr (sizeof(T) == 4) v = reinterpret_cast<const float*>(x)[t];
@@ -189,12 +277,14 @@ struct Quant1DArgs {
   int64_t rb_upper;        // row-blocks covered by the launch (grouped: upper bound)
   int64_t ct_count;        // column tiles = atoms along columns
   unsigned* status;
+  const uint32_t* rbits;   // kQuantSR: one random word per element, row-major [rows, cols]
+  uint32_t signs;          // kQuantRHT: the 16 sign bits of the transform
 };
 
 // One tile = 128 rows x (4 * BLOCK) columns = exactly one 512-byte scale atom.
 // 256 threads; each thread owns one 16-byte chunk per pass; the lanes of one block
 // (BLOCK / elements-per-chunk of them, adjacent) combine their maxima by shuffles.
-template <typename T, int BLOCK, bool MX, bool HW>
+template <typename T, int BLOCK, bool MX, bool HW, int VAR = kQuantPlain>
 __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int EPC = Elem<T>::kPerChunk;
   constexpr int TC = 4 * BLOCK;             // columns per tile
@@ -203,6 +293,9 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int PASSES = 128 / RPP;
   constexpr int LPB = BLOCK / EPC;          // lanes per block
   static_assert(EPC == 4 || EPC == 8, "chunk");
+  static_assert(VAR != kQuantMxFloor || MX, "the rounded-down scale is an E8M0 one");
+  static_assert(VAR != kQuantSR || (!MX && BLOCK == 16), "stochastic rounding: NVFP4");
+  constexpr int RW = VAR == kQuantSR ? EPC / 4 : 0;  // 16-byte loads of random words per chunk
 
   __shared__ __align__(16) uint8_t s_sf[512];
   __shared__ int s_rb[kMaxGroups + 1];
@@ -257,6 +350,7 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
     const bool col_ok = col < p.cols;
 
     uint4 u[PASSES];
+    uint4 rw[PASSES][RW > 0 ? RW : 1];
 #pragma unroll
     for (int ps = 0; ps < PASSES; ++ps) {
       const int64_t r = row_base + ps * RPP + tid / CPR;
@@ -264,6 +358,11 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
         u[ps] = ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + col) * sizeof(T));
       else
         u[ps] = make_uint4(0, 0, 0, 0);
+      if constexpr (RW > 0) {
+#pragma unroll
+        for (int j = 0; j < RW; ++j)
+          rw[ps][j] = (col_ok && r < row_end) ? ld_stream(p.rbits + r * p.cols + col + 4 * j) : make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
     for (int ps = 0; ps < PASSES; ++ps) {
@@ -271,6 +370,7 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       const int64_t r = row_base + rl;
       float v[EPC];
       Elem<T>::unpack(u[ps], v);
+      if constexpr (VAR == kQuantRHT) rht16_lanes<EPC>(v, p.signs, (chunk % (16 / EPC)) * EPC);
       uint32_t m = 0;
 #pragma unroll
       for (int i = 0; i < EPC; ++i) m = max(m, abs_bits(v[i]));
@@ -281,7 +381,7 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       uint32_t sb;
       float mul;
       if constexpr (MX) {
-        sb = e8m0_code(__fdiv_rn(amax_b, 6.0f));
+        sb = VAR == kQuantMxFloor ? e8m0_floor_code(amax_b) : e8m0_code(__fdiv_rn(amax_b, 6.0f));
         mul = e8m0_inverse(sb);
       } else {
         mul = nvfp4_block_scale(amax_b, g, sb);
@@ -297,7 +397,20 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
         }
       }
       const bool ok = col_ok && r < row_end;
-      if constexpr (EPC == 8) {
+      if constexpr (VAR == kQuantSR) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < EPC; ++i) {
+          const uint4 w4 = rw[ps][i / 4];
+          const uint32_t bits = (i & 3) == 0 ? w4.x : (i & 3) == 1 ? w4.y : (i & 3) == 2 ? w4.z : w4.w;
+          packed |= e2m1_code_sr(s[i], bits) << (4 * i);
+        }
+        if constexpr (EPC == 8) {
+          if (ok) *reinterpret_cast<uint32_t*>(p.codes + r * half_cols + col / 2) = packed;
+        } else {
+          if (ok) *reinterpret_cast<uint16_t*>(p.codes + r * half_cols + col / 2) = static_cast<uint16_t>(packed);
+        }
+      } else if constexpr (EPC == 8) {
         const uint32_t packed = pack8<HW>(s);
         if (ok) *reinterpret_cast<uint32_t*>(p.codes + r * half_cols + col / 2) = packed;
       } else {
@@ -621,6 +734,14 @@ __global__ void debug_encode_kernel(const float* in, int64_t n, int which, uint8
 
 __global__ void set_value_kernel(float* p, float v) { *p = v; }
 
+__global__ void global_scale_kernel(const float* amax, float* g, unsigned* status) {
+  allow_dependents();
+  wait_prior_grids();  // the maximum may come from the kernel (or collective) just before
+  const float a = *amax;
+  if (!(abs_bits(a) < 0x7F800000u)) atomicOr(status, kStatusNonFinite);
+  *g = a > 0.0f ? __fdiv_rn(a, 2688.0f) : 1.0f;  // 2688 = 6 * 448
+}
+
 // ------------------------------------------------------------------ launchers
 static int blocks_for(int64_t work, int per_sm) {
   const int sms = num_sms();
@@ -629,7 +750,7 @@ static int blocks_for(int64_t work, int per_sm) {
 }
 
 cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float* amax_out, float* g_out,
-                        unsigned* status, cudaStream_t st) {
+                        unsigned* status, cudaStream_t st, int rht, uint32_t signs) {
   const int epc = bf16 ? 8 : 4;
   const int64_t chunks = (n + epc - 1) / epc;
   int blocks = static_cast<int>(std::min<int64_t>((chunks + 2047) / 2048, static_cast<int64_t>(num_sms()) * 4));
@@ -643,13 +764,21 @@ cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float*
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (rht) {
+    if (bf16)
+      return cudaLaunchKernelEx(&cfg, amax_kernel<__nv_bfloat16, true>, static_cast<const __nv_bfloat16*>(x), n, ws,
+                                amax_out, g_out, status, signs);
+    return cudaLaunchKernelEx(&cfg, amax_kernel<float, true>, static_cast<const float*>(x), n, ws, amax_out, g_out,
+                              status, signs);
+  }
   if (bf16)
     return cudaLaunchKernelEx(&cfg, amax_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x), n, ws, amax_out,
-                              g_out, status);
-  return cudaLaunchKernelEx(&cfg, amax_kernel<float>, static_cast<const float*>(x), n, ws, amax_out, g_out, status);
+                              g_out, status, 0u);
+  return cudaLaunchKernelEx(&cfg, amax_kernel<float>, static_cast<const float*>(x), n, ws, amax_out, g_out, status,
+                            0u);
 }
 
-template <typename T, int BLOCK, bool MX>
+template <typename T, int BLOCK, bool MX, int VAR = kQuantPlain>
 static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
   const int blocks = blocks_for(a.rb_upper * a.ct_count, 8);
   cudaLaunchConfig_t cfg = {};
@@ -661,12 +790,13 @@ static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware>, a);
+  return cudaLaunchKernelEx(&cfg, quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware, VAR>, a);
 }
 
 cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
                                uint8_t* scales, const float* g, const int32_t* offsets, int num_groups,
-                               unsigned* status, cudaStream_t st) {
+                               unsigned* status, cudaStream_t st, int variant, const uint32_t* rbits,
+                               uint32_t signs) {
   Quant1DArgs a;
   a.x = x;
   a.rows = rows;
@@ -680,7 +810,24 @@ cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf
   const int blk = mx ? 32 : 16;
   a.ct_count = ((cols / blk) + 3) / 4;
   a.status = status;
-  if (bf16) return mx ? launch_q1d_t<__nv_bfloat16, 32, true>(a, st) : launch_q1d_t<__nv_bfloat16, 16, false>(a, st);
+  a.rbits = rbits;
+  a.signs = signs;
+  using BF = __nv_bfloat16;
+  switch (variant) {
+    case kQuantMxFloor:
+      if (!mx) return cudaErrorInvalidValue;
+      return bf16 ? launch_q1d_t<BF, 32, true, kQuantMxFloor>(a, st) : launch_q1d_t<float, 32, true, kQuantMxFloor>(a, st);
+    case kQuantSR:
+      if (mx) return cudaErrorInvalidValue;
+      return bf16 ? launch_q1d_t<BF, 16, false, kQuantSR>(a, st) : launch_q1d_t<float, 16, false, kQuantSR>(a, st);
+    case kQuantRHT:
+      if (bf16)
+        return mx ? launch_q1d_t<BF, 32, true, kQuantRHT>(a, st) : launch_q1d_t<BF, 16, false, kQuantRHT>(a, st);
+      return mx ? launch_q1d_t<float, 32, true, kQuantRHT>(a, st) : launch_q1d_t<float, 16, false, kQuantRHT>(a, st);
+    default:
+      break;
+  }
+  if (bf16) return mx ? launch_q1d_t<BF, 32, true>(a, st) : launch_q1d_t<BF, 16, false>(a, st);
   return mx ? launch_q1d_t<float, 32, true>(a, st) : launch_q1d_t<float, 16, false>(a, st);
 }
 
@@ -757,6 +904,19 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
 cudaError_t launch_set_value(float* p, float v, cudaStream_t st) {
   set_value_kernel<<<1, 1, 0, st>>>(p, v);
   return cudaGetLastError();
+}
+
+cudaError_t launch_global_scale(const float* amax, float* g, unsigned* status, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, global_scale_kernel, amax, g, status);
 }
 
 cudaError_t launch_debug_encode(const float* in, int64_t n, int which, uint8_t* out, cudaStream_t st) {

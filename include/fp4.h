@@ -121,6 +121,56 @@ fp4_status fp4_quantize_grouped(const void* x_dev, int64_t rows, int64_t cols, f
                                 float* global_out_dev, const float* global_in_dev,
                                 void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* fp4_quantize with options ("MXFP4 / NVFP4 video transcript", MXFP4 passage: a scale
+ * that is not a power of two must be rounded to one, 70 to 64 or 128).  flags:
+ *   FP4_QUANT_E8M0_FLOOR  (MXFP4 only) round the block scale down instead of to nearest:
+ *       sb = 2^(floor(log2 amax_b) - 2), the largest power of two not above amax_b divided
+ *       by 4 (E2M1's largest power of two), code clamped to [0, 254].  The block's largest
+ *       element then scales into [4, 8); values from 6 up saturate to 6.
+ * Other arguments and errors as fp4_quantize; unknown bits return FP4_ERR_INVALID_ARG. */
+#define FP4_QUANT_E8M0_FLOOR 1u
+fp4_status fp4_quantize_ex(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
+                           int block, unsigned flags, uint8_t* codes_out_dev, uint8_t* scales_out_dev,
+                           float* global_out_dev, uint8_t* codesT_out_dev, uint8_t* scalesT_out_dev,
+                           const float* global_in_dev, void* workspace_dev, size_t workspace_bytes,
+                           void* stream);
+
+/* NVFP4 1-D quantization with stochastic rounding of the elements ("MXFP4 / NVFP4 video
+ * transcript", training-recipe passage: 0.3 between 0 and 1 becomes 1 with probability
+ * 0.3, so that the expected value is kept; used for gradients).  The global and block
+ * scales are fp4_quantize's; only the element rounding changes: a scaled magnitude a
+ * between grid neighbours lo < a < hi becomes hi iff u < (a - lo) / (hi - lo), with
+ * u = (rbits[i] >> 8) * 2^-24; grid values stay, a >= 6 saturates, the sign is kept.
+ *   rbits_dev  one uint32 random word per element, row-major [rows, cols], 16-byte
+ *              aligned (the caller draws them).
+ * Other arguments and errors as fp4_quantize (block 16). */
+fp4_status fp4_quantize_sr(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype,
+                           const uint32_t* rbits_dev, uint8_t* codes_out_dev, uint8_t* scales_out_dev,
+                           float* global_out_dev, const float* global_in_dev, void* workspace_dev,
+                           size_t workspace_bytes, void* stream);
+
+/* Quantization after a 16-point random Hadamard transform ("MXFP4 / NVFP4 video
+ * transcript", training-recipe passage; "FP4" glossary entry, "Inference and training in
+ * FP4": outliers are spread over their block before quantizing).  Every 16-element block
+ * b along cols becomes (1/4) H16 diag(s) b, H16 the Sylvester Hadamard matrix and
+ * s_j = -1 where bit j of `signs` (16 bits) is set, computed in FP32 as the signs, the
+ * butterfly stages of half-width 1, 2, 4, 8, then the factor 1/4; the transformed tensor
+ * is then quantized as fp4_quantize does (NVFP4 block 16, g from the transformed tensor's
+ * amax unless global_in_dev is given; or MXFP4 block 32).  Both operands of a GEMM
+ * transformed with the same signs keep their products: Q is orthogonal. */
+fp4_status fp4_quantize_rht(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype, fp4_fmt fmt,
+                            uint32_t signs, uint8_t* codes_out_dev, uint8_t* scales_out_dev,
+                            float* global_out_dev, const float* global_in_dev, void* workspace_dev,
+                            size_t workspace_bytes, void* stream);
+
+/* NVFP4 global scale from a tensor amax already on the device ("MXFP4 / NVFP4 video
+ * transcript", NVFP4 passage): global_out_dev[0] = amax / (6 * 448), or 1 for amax = 0.
+ * For tensors split over ranks: each rank's fp4_amax, one all-reduce (MAX) of that float,
+ * then this call gives every rank the g of the whole tensor, and fp4_quantize with
+ * global_in_dev = g quantizes each shard exactly as the whole tensor would be.  A
+ * non-finite amax latches FP4_ERR_NONFINITE. */
+fp4_status fp4_global_scale(const float* amax_dev, float* global_out_dev, void* stream);
+
 /* Dequantize (debug / tests): out_dev[r, k] = E2M1(code) * dec(scale) * g as FP32, for a
  * [rows, cols] tensor in the layouts above; global_dev may be NULL (g = 1). */
 fp4_status fp4_dequantize(const uint8_t* codes_dev, const uint8_t* scales_dev,
@@ -158,6 +208,28 @@ fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev,
                        const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
                        int64_t M, int64_t N, int64_t K, void* D_dev, fp4_dtype out_dtype,
                        void* workspace_dev, size_t workspace_bytes, unsigned flags, void* stream);
+
+/* GEMM with the epilogue that follows the scale ("Rubin FP4 GEMM overview" 3.2: the FP32
+ * result is multiplied by the scale factors, the bias is added, the activation applied,
+ * then it is converted to the output format, FP4 included; 4.2: C = (A.B)(sA.sB) + bias):
+ *   t[m, n] = act(gA gB sum_k ... + bias[n])      (FP32: product, then + bias, then act)
+ *   D_dev   [M, N] in out_dtype (BF16 round to nearest even, or FP32), or NULL;
+ *   Dcodes_dev / Dscales_dev: or an NVFP4 copy of t (or both): 16-element blocks along n,
+ *           codes [M, N/2], scales fp4_scales_bytes(M, N, FP4_NVFP4) in the swizzled
+ *           layout, quantized exactly as fp4_quantize would quantize the FP32 t with
+ *           global_in = gD_dev (the caller's global scale: t's amax is not known until
+ *           the whole product is, so it cannot be computed here).  The result can feed
+ *           the next fp4_gemm as its A operand directly.  Needs N % 32 == 0.
+ *   bias_dev [N] FP32 or NULL; act FP4_ACT_NONE or FP4_ACT_RELU.
+ * workspace: fp4_gemm_epilogue_workspace_size(M, N, K, fmt, Dcodes_dev != NULL) bytes,
+ * zero-filled before first use (left zero-filled).  Plain (not grouped) problems only. */
+typedef enum { FP4_ACT_NONE = 0, FP4_ACT_RELU = 1 } fp4_act;
+size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int fp4_out);
+fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,
+                             const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
+                             int64_t M, int64_t N, int64_t K, const float* bias_dev, fp4_act act,
+                             void* D_dev, fp4_dtype out_dtype, uint8_t* Dcodes_dev, uint8_t* Dscales_dev,
+                             const float* gD_dev, void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /* BF16-activation GEMM (quantize-on-load): D = gX * gB * (Xq . Bq^T) where Xq is the
  * NVFP4 quantization of the bf16 activations X [M, K] (tensor amax -> gX, 16-blocks,

@@ -67,3 +67,68 @@ def test_single_process_defaults():
     d.barrier()
     d.close()
     assert bench.whole_job_value(10.0, 1, 2.0) == pytest.approx(5000.0)
+
+
+# ---------------------------------------------------------------- row-sharded quantization
+def _shard_main(rank: int, world: int, port: int, x, splits, results):
+    """Each rank: the oracle's amax of its rows, the library's reduce_amax_ over gloo,
+    then the oracle's quantization of its rows with the reduced tensor's g."""
+    import numpy as np
+    import oracle
+    import torch
+    import torch.distributed as dist
+
+    from block_scaled_fp4_04_b200 import sharded
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        lo, hi = splits[rank], splits[rank + 1]
+        local = np.ascontiguousarray(x[lo:hi])
+        amax = torch.tensor([oracle.amax(local)], dtype=torch.float32)
+        sharded.reduce_amax_(amax)
+        g = oracle.global_scale(float(amax.item()))
+        q = oracle.quantize(local, oracle.NVFP4, 16, g_in=g)
+        results[rank] = (float(amax.item()), q["codes"].tobytes(), q["scales"].tobytes(), float(g))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("splits", [[0, 40, 96], [0, 95, 96]])
+def test_row_shards_with_one_max_all_reduce_equal_the_whole_tensor(splits):
+    """Two gloo ranks hold row shards of one tensor (the largest element on one of them);
+    after the all-reduce (MAX) of their local maxima, each rank's quantization equals the
+    whole tensor's rows bit for bit, and both ranks hold the same g."""
+    import numpy as np
+    import oracle
+    world = len(splits) - 1
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((splits[-1], 256)).astype(np.float32)
+    x[splits[1], 7] = 60.0              # the tensor amax sits on rank 1
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    results = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_main, args=(r, world, port, x, splits, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    whole = oracle.quantize(x, oracle.NVFP4, 16)
+    for r in range(world):
+        amax, codes, scales, g = results[r]
+        lo, hi = splits[r], splits[r + 1]
+        assert amax == 60.0
+        assert np.float32(g) == whole["g"]
+        assert codes == whole["codes"][lo:hi].tobytes()
+        assert scales == whole["scales"][lo:hi].tobytes()
+    # without the exchange rank 0 would pick its own, smaller g and different scales
+    local0 = oracle.quantize(np.ascontiguousarray(x[:splits[1]]), oracle.NVFP4, 16)
+    assert local0["g"] != whole["g"]
+
+
+def test_reduce_amax_is_a_no_op_without_a_process_group():
+    import torch
+    from block_scaled_fp4_04_b200 import sharded
+    t = torch.tensor([2.5])
+    assert sharded.reduce_amax_(t).item() == 2.5
