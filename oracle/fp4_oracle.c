@@ -218,6 +218,16 @@ static double e8m0_value(int c) {
     return e8m0_table[c];
 }
 
+/* Builds the three code tables before rows are processed on several threads (each
+ * table is filled on first use; filling it once up front keeps the threads from doing
+ * it concurrently).  Rows are independent, so running them on OpenMP threads changes
+ * no arithmetic. */
+static void tables_ready(void) {
+    (void)e2m1_magnitude(0);
+    (void)e4m3_value(0);
+    (void)e8m0_value(0);
+}
+
 /* v >= 0.  Nearest power of two 2^(c-127), c in 0..254, in the linear domain; an
  * exact midpoint (1.5 * 2^e) goes to the larger power. */
 uint8_t orc_e8m0_encode(float v) {
@@ -336,10 +346,12 @@ int orc_quantize_nvfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype
     if (orc_amax(x, rows * cols, dtype, &amax_t) != ORC_OK) return ORC_ERR_NONFINITE;
     g = g_in ? *g_in : orc_global_scale(amax_t);
     if (g_out) *g_out = g;
-    float xs[16];
-    uint8_t cb[16];
-    uint8_t* row_codes = (uint8_t*)malloc((size_t)cols);
+    tables_ready();
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
+        float xs[16];
+        uint8_t cb[16];
+        uint8_t* row_codes = (uint8_t*)malloc((size_t)cols);
         for (int64_t b = 0; b < cols / 16; ++b) {
             float amax_b = 0.0f;
             for (int i = 0; i < 16; ++i) {
@@ -351,8 +363,8 @@ int orc_quantize_nvfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype
             memcpy(row_codes + b * 16, cb, 16);
         }
         pack_row(row_codes, cols, codes + r * (cols / 2));
+        free(row_codes);
     }
-    free(row_codes);
     return ORC_OK;
 }
 
@@ -373,23 +385,27 @@ int orc_quantize_mxfp4_1d(const void* x, int64_t rows, int64_t cols, int dtype,
  * orc_e8m0_encode_floor). */
 int orc_quantize_mxfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype, int floor_mode,
                             uint8_t* codes, uint8_t* scales_rm) {
-    float xs[32];
-    uint8_t cb[32];
-    uint8_t* row_codes = (uint8_t*)malloc((size_t)cols);
+    /* a non-finite element anywhere is an error (no encoding exists for it) */
+    for (int64_t i = 0; i < rows * cols; ++i)
+        if (!isfinite(load_elem(x, i, dtype))) return ORC_ERR_NONFINITE;
+    tables_ready();
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
+        float xs[32];
+        uint8_t cb[32];
+        uint8_t* row_codes = (uint8_t*)malloc((size_t)cols);
         for (int64_t b = 0; b < cols / 32; ++b) {
             float amax_b = 0.0f;
             for (int i = 0; i < 32; ++i) {
                 xs[i] = load_elem(x, r * cols + b * 32 + i, dtype);
-                if (!isfinite(xs[i])) { free(row_codes); return ORC_ERR_NONFINITE; }
                 if (fabsf(xs[i]) > amax_b) amax_b = fabsf(xs[i]);
             }
             scales_rm[r * (cols / 32) + b] = mxfp4_encode_block(xs, 32, amax_b, floor_mode, cb);
             memcpy(row_codes + b * 32, cb, 32);
         }
         pack_row(row_codes, cols, codes + r * (cols / 2));
+        free(row_codes);
     }
-    free(row_codes);
     return ORC_OK;
 }
 
@@ -409,9 +425,11 @@ int orc_quantize_nvfp4_2d(const void* x, int64_t rows, int64_t cols, int dtype, 
     g = g_in ? *g_in : orc_global_scale(amax_t);
     if (g_out) *g_out = g;
     uint8_t* full = (uint8_t*)malloc((size_t)(rows * cols)); /* unpacked codes of W */
-    float xs[256];
-    uint8_t cb[256];
+    tables_ready();
+#pragma omp parallel for schedule(static)
     for (int64_t tr = 0; tr < rows / 16; ++tr) {
+        float xs[256];
+        uint8_t cb[256];
         for (int64_t tc = 0; tc < cols / 16; ++tc) {
             float amax_b = 0.0f;
             for (int i = 0; i < 16; ++i)
@@ -430,12 +448,13 @@ int orc_quantize_nvfp4_2d(const void* x, int64_t rows, int64_t cols, int dtype, 
         }
     }
     for (int64_t r = 0; r < rows; ++r) pack_row(full + r * cols, cols, codes + r * (cols / 2));
-    uint8_t* colbuf = (uint8_t*)malloc((size_t)rows);
+#pragma omp parallel for schedule(static)
     for (int64_t c = 0; c < cols; ++c) {
+        uint8_t* colbuf = (uint8_t*)malloc((size_t)rows);
         for (int64_t r = 0; r < rows; ++r) colbuf[r] = full[r * cols + c];
         pack_row(colbuf, rows, codesT + c * (rows / 2));
+        free(colbuf);
     }
-    free(colbuf);
     free(full);
     return ORC_OK;
 }
@@ -503,6 +522,8 @@ void orc_swizzle_scales_grouped(const uint8_t* rm, const int32_t* offsets, int n
 void orc_dequantize(const uint8_t* codes, const uint8_t* scales_rm, float g, int64_t rows, int64_t cols,
                     int fmt, double* out) {
     int blk = fmt == 0 ? 16 : 32;
+    tables_ready();
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t k = 0; k < cols; ++k) {
             uint8_t byte = codes[r * (cols / 2) + k / 2];
