@@ -8,8 +8,11 @@ amax + NVFP4 quantize of the activations + the FP4 GEMM.  Memory-bound, so the m
 is GB/s of algorithmic bytes (each operand's stored bytes read once, output written
 once; the activations are read twice, once for the amax and once for the encode).
 
-Other workloads (--workload prefill | moe | train | quantize) measure the remaining
-configurations the same way.
+The same JSON line carries a sub-record for each other configuration (prefill 8192^3 with
+BF16 activations quantized every step; the training step at S = 16384; the MXFP4 grouped
+MoE GEMM; the quantize kernels alone), each with its roofline, its own clock sample, an
+end-to-end figure with host buffers and the oracle's rate on a bounded sample.
+--workload prefill | moe | train | quantize prints one of them alone.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload ...]
 
@@ -229,26 +232,36 @@ def run_decode(args, dist: Dist, dev):
     if fp4.fp4_get_status() != fp4.OK:
         raise RuntimeError("device status latched an error during warm-up")
 
+    # Timed region: exactly K steps between a barrier and a synchronize on both sides,
+    # repeated back to back until at least half a second of timed work, so that the clock
+    # samples cover what is measured; the reported time is the median batch (each batch's
+    # time the maximum over ranks).  Every rank runs the same number of batches.
     K = args.steps
     clocks = ClockSampler(dev.index or 0)
     time.sleep(0.15)
-    dist.barrier()
-    torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    batch_ms, total_ms = [], 0.0
     c0 = clocks.mark()
-    t_start.record()
-    for i in range(K):
-        step(i)
-    t_end.record()
-    torch.cuda.synchronize()
-    dist.barrier()
+    while True:
+        dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record()
+        for i in range(K):
+            step(i)
+        t_end.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        b = dist.max(t_start.elapsed_time(t_end), dev)
+        batch_ms.append(b)
+        total_ms += b
+        if total_ms >= 500.0 and len(batch_ms) >= 3:
+            break
     c1 = clocks.mark()
-    ms = t_start.elapsed_time(t_end)
     clk = clocks.stop(c0, c1)
     if fp4.fp4_get_status() != fp4.OK:
         raise RuntimeError("device status latched an error during the timed steps")
-    max_ms = dist.max(ms, dev)
+    max_ms = statistics.median(batch_ms)
 
     # The step is one launch of one kernel, so the events around the timed batch give its
     # average launch duration.  For reference, the same GEMM on pre-quantized activations
@@ -301,6 +314,9 @@ def run_decode(args, dist: Dist, dev):
         "n_gpus": dist.world,
         "steps": K,
         "warmup": args.warmup,
+        "batches": len(batch_ms),
+        "timing": f"median of {len(batch_ms)} back-to-back batches of exactly {K} steps, each between a barrier "
+                  "and a synchronize, max over ranks",
         "ms_per_step": max_ms / K,
         "higher_is_better": True,
         "scaling": "weak",
@@ -335,22 +351,9 @@ def run_decode(args, dist: Dist, dev):
     return res
 
 
-# ---------------------------------------------------------------- other workloads
+# ---------------------------------------------------------------- the other configurations
 FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
-
-
-def _events_ms(fn, iters: int, warmup: int) -> float:
-    """Average device ms per call of fn(i), events around a batch on the current stream."""
-    for i in range(warmup):
-        fn(i)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(iters):
-        fn(i)
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / iters
+MIN_TIMED_S = 0.4   # each sub-workload is timed over at least this long (clock samples cover it)
 
 
 def _check(fp4):
@@ -363,22 +366,110 @@ def _copies(per_copy_bytes: int) -> int:
     return max(1, int(np.ceil(3 * L2_BYTES / max(per_copy_bytes, 1))))
 
 
-def _line(workload: str, value, unit: str, ms: float, args, extra: dict) -> dict:
-    res = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "data": "synthetic (seeded, same recipes as the tests)", "config": {"workload": workload}}
-    res.update(extra)
-    return res
+def timed_batches(fn, steps: int, warmup: int, dev_index: int, min_s: float = MIN_TIMED_S):
+    """Warm-up, then back-to-back batches of `steps` calls of fn(i), each batch bracketed by
+    CUDA events on the current stream, until at least min_s of timed work; returns the
+    median ms per call over the batches, the batches, and the clocks sampled meanwhile."""
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev_index)
+    time.sleep(0.15)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    batches, total, i = [], 0.0, 0
+    c0 = clocks.mark()
+    while total < min_s * 1e3 or len(batches) < 3:
+        e0.record()
+        for _ in range(steps):
+            fn(i)
+            i += 1
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        batches.append(ms / steps)
+        total += ms
+    c1 = clocks.mark()
+    clk = clocks.stop(c0, c1)
+    return statistics.median(batches), batches, clk
 
 
-def run_prefill(args, dev):
-    """Prefill-shaped NVFP4 GEMM 8192^3: BF16 activations quantized every step (tensor amax,
-    then 16-blocks), weights pre-quantized; tensor-bound."""
+def mma_peak(dev) -> dict:
+    """The block-scaled MMA loop's throughput on every SM (library probe fp4_mma_peak)."""
+    import block_scaled_fp4_04_b200 as fp4
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    cyc = torch.zeros(sms, dtype=torch.int64, device=dev)
+    iters = 20000
+    fp4.fp4_mma_peak(iters, sms, cyc)  # warm
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fp4.fp4_mma_peak(iters, sms, cyc)
+    e1.record()
+    torch.cuda.synchronize()
+    _check(fp4)
+    ms = e0.elapsed_time(e1)
+    flop = 2.0 * 128 * 256 * 64 * 4 * iters
+    c = float(cyc.double().mean().item())
+    return {"TFLOP/s": flop * sms / (ms * 1e-3) / 1e12, "flop_per_clk_per_sm": flop / c,
+            "sm_ghz": c / (ms * 1e-3) / 1e9, "probe": "fp4_mma_peak: 4 x tcgen05.mma.kind::mxf4nvf4 "
+            "M=128 N=256 K=64 per K step from shared memory, no loads, one CTA per SM"}
+
+
+def _tensor_roofline(kernel: str, flop: float, ms: float, peaks: dict, traffic_key: str, extra=None) -> dict:
+    achieved = flop / (ms * 1e-3) / 1e12
+    r = {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peaks["fp4"], "unit": "TFLOP/s",
+         "frac": achieved / peaks["fp4"], "peak_source": peaks["fp4_source"], "launch_ms": ms,
+         "frac_of_mma_loop": achieved / peaks["mma_loop"] if peaks.get("mma_loop") else None,
+         "frac_of_nominal_9pf": achieved / 9000.0, "traffic": traffic_for(traffic_key)}
+    if extra:
+        r.update(extra)
+    return r
+
+
+def _e2e(step_on, host_in: list, dev_in: list, host_out: list, dev_out: list, steps: int, warmup: int) -> float:
+    """ms per step through the library with host buffers: every step copies the inputs from
+    pinned host memory, runs the step, and reads the outputs back."""
+    def one(i):
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        step_on(i)
+        for h, d in zip(host_out, dev_out):
+            h.copy_(d, non_blocking=True)
+    ms, _, _ = timed_batches(one, max(1, min(steps, 20)), min(warmup, 3), torch.cuda.current_device(), min_s=0.2)
+    return ms
+
+
+def _oracle_rows_gemm_rate(x_rows: np.ndarray, fmt: int, blk: int, w_hat: np.ndarray, g=None, budget_s=4.0):
+    """The oracle, as it stands, on a sample: quantize the given activation rows and take
+    their FP64 product with the (already dequantized) weights; returns TFLOP/s of the
+    sampled rows, the threads used, and the repetitions."""
+    import oracle
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        q = oracle.quantize(x_rows, fmt, blk, g_in=g)
+        a_hat = oracle.dequantize(q["codes"], q["scales"], q["g"], fmt)
+        oracle.gemm_reference(a_hat, w_hat)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    flop = 2.0 * x_rows.shape[0] * w_hat.shape[0] * w_hat.shape[1] * reps
+    return flop / dt / 1e12, oracle.num_threads(), reps
+
+
+def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
+    """Prefill-shaped NVFP4 GEMM 8192^3: BF16 activations (0.1% outliers x50) quantized every
+    step (tensor amax, then 16-blocks), weights pre-quantized; BF16 out; tensor-bound."""
     import block_scaled_fp4_04_b200 as fp4
     m = n = k = 8192
     x, w = workloads.prefill_inputs(device="cpu")
-    x = x.to(dev)
-    qw = fp4.quantize(w.to(dev), fp4.NVFP4, 16)
+    xd = x.to(dev)
+    per_copy = n * k // 2 + fp4.fp4_scales_bytes(n, k, fp4.NVFP4)
+    copies = _copies(per_copy)
+    w_dev = w.to(dev)
+    wq = [fp4.quantize(w_dev, fp4.NVFP4, 16) for _ in range(copies)]
+    del w_dev
     L = fp4.lib()
     P = lambda t: t.data_ptr()
     xc = torch.empty(m, k // 2, dtype=torch.uint8, device=dev)
@@ -389,44 +480,131 @@ def run_prefill(args, dev):
     d = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
     sp = torch.cuda.current_stream().cuda_stream
 
-    def step(i):
-        if L.fp4_gemm_bf16a(P(x), P(qw.codes), P(qw.scales), P(qw.g), m, n, k, P(d), fp4.BF16, P(xc), P(xs),
-                            P(xg), P(ws), wn, fp4.GEMM_WEIGHTS_READY, sp):
+    def step(i, src=None):
+        q = wq[i % copies]
+        if L.fp4_gemm_bf16a(P(src if src is not None else xd), P(q.codes), P(q.scales), P(q.g), m, n, k, P(d),
+                            fp4.BF16, P(xc), P(xs), P(xg), P(ws), wn, fp4.GEMM_WEIGHTS_READY, sp):
             raise RuntimeError(fp4.fp4_last_error())
 
     def gemm(i):
-        if L.fp4_gemm_ex(fp4.NVFP4, P(xc), P(xs), P(xg), P(qw.codes), P(qw.scales), P(qw.g), m, n, k, P(d),
-                         fp4.BF16, P(ws), wn, 0, sp):
+        q = wq[i % copies]
+        if L.fp4_gemm_ex(fp4.NVFP4, P(xc), P(xs), P(xg), P(q.codes), P(q.scales), P(q.g), m, n, k, P(d), fp4.BF16,
+                         P(ws), wn, 0, sp):
             raise RuntimeError(fp4.fp4_last_error())
 
-    step_ms = _events_ms(step, args.steps, args.warmup)
-    gemm_ms = _events_ms(gemm, args.steps, args.warmup)
+    di = dev.index or 0
+    step_ms, batches, clk = timed_batches(step, args.steps, args.warmup, di)
+    gemm_ms, _, gclk = timed_batches(gemm, args.steps, args.warmup, di)
     _check(fp4)
     flop = 2.0 * m * n * k
-    hbm, bf16, bf16_s, src = load_peaks()
-    peak = bf16 * FP4_PER_BF16
-    gemm_tf = flop / (gemm_ms * 1e-3) / 1e12
-    step_tf = flop / (step_ms * 1e-3) / 1e12
-    return _line("prefill-shaped NVFP4 GEMM M=N=K=8192, bf16 activations quantized every step, bf16 out",
-                 step_tf, "TFLOP/s", step_ms, args, {
-                     "dtype": "nvfp4 x nvfp4 -> fp32 accumulate, bf16 out",
-                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1, CTA pair>",
-                                  "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s", "frac": gemm_tf / peak,
-                                  "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)",
-                                  "frac_of_nominal_9pf": gemm_tf / 9000.0, "launch_ms": gemm_ms,
-                                  "traffic": None},
-                     "step": {"ms": step_ms, "TFLOP/s": step_tf, "contents": "amax + quantize(X) + GEMM"},
-                     "gpu_launches": 3 * args.steps})
+    x_host = x.pin_memory()
+    d_host = torch.empty(m, n, dtype=torch.bfloat16).pin_memory()
+    x_stage = torch.empty_like(xd)
+    e2e_ms = _e2e(lambda i: step(i, x_stage), [x_host], [x_stage], [d_host], [d], args.steps, args.warmup)
+    _check(fp4)
+    rec = {"value": flop / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms,
+           "steps_per_batch": args.steps, "batches": len(batches), "timing": "median over batches",
+           "config": {"workload": "prefill-shaped NVFP4 GEMM M=N=K=8192, bf16 activations (0.1% outliers x50) "
+                                  "quantized every step, weights N(0,0.02) pre-quantized, bf16 out",
+                      "step": "fp4_gemm_bf16a: tensor amax + NVFP4 quantize of X + FP4 GEMM (3 launches)",
+                      "l2": f"weights rotate over {copies} pre-quantized copies "
+                            f"({copies * per_copy / 2**20:.0f} MiB); X (128 MiB) exceeds the L2"},
+           "roofline": _tensor_roofline("fp4_gemm_kernel<256, nvfp4, 1 acc, CTA pair>", flop, gemm_ms, peaks,
+                                        "prefill_gemm", {"gemm_clocks": gclk}),
+           "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                   "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2},
+           "gpu_launches_per_step": 3, "clocks": clk}
+    if cpu:
+        import oracle
+        rows = 8
+        xb = workloads.bf16_bits(x)
+        g = oracle.global_scale(oracle.amax(xb))
+        ow = oracle.quantize(w.numpy(), oracle.NVFP4, 16)
+        w_hat = oracle.dequantize(ow["codes"], ow["scales"], ow["g"])
+        v, cores, reps = _oracle_rows_gemm_rate(np.ascontiguousarray(xb[:rows]), oracle.NVFP4, 16, w_hat, g)
+        rec["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{reps} x (quantize {rows} rows of X with the tensor's g, FP64 product "
+                                         f"with the 8192 x 8192 dequantized weights)"}
+    del wq, xd, xc, xs, ws, d, x_stage
+    torch.cuda.empty_cache()
+    return rec
 
 
-def run_moe(args, dev):
-    """MXFP4 grouped MoE GEMM: 4096 tokens x top-4 of 32 experts, K=2880, N=5760; the
-    activations are quantized (grouped layout) every step."""
+def measure_train(args, dev, peaks, cpu: bool, s: int = 16384) -> dict:
+    """Training-recipe step at S: W quantized once with 16x16 blocks (W and W^T); per step X
+    and dY quantized (16-blocks), forward D = X W^T and backward dX = dY W, bf16 out."""
+    import block_scaled_fp4_04_b200 as fp4
+    x, w, dy = workloads.train_inputs(s, device="cpu")
+    xd, dyd = x.to(dev), dy.to(dev)
+    qw = fp4.quantize(w.to(dev), fp4.NVFP4, 256)
+    wt = fp4.transposed(qw)
+    ws = fp4.Workspace(dev)
+    dout = torch.empty(s, s, dtype=torch.bfloat16, device=dev)
+    dxout = torch.empty(s, s, dtype=torch.bfloat16, device=dev)
+    state = {}
+
+    def step(i, xs=None, dys=None):
+        qx = fp4.quantize(xs if xs is not None else xd, fp4.NVFP4, 16, workspace=ws)
+        qd = fp4.quantize(dys if dys is not None else dyd, fp4.NVFP4, 16, workspace=ws)
+        fp4.gemm(qx, qw, out=dout, workspace=ws)
+        fp4.gemm(qd, wt, out=dxout, workspace=ws)
+        state["qx"], state["qd"] = qx, qd
+
+    di = dev.index or 0
+    steps = max(3, args.steps // 4)
+    step_ms, batches, clk = timed_batches(step, steps, args.warmup, di)
+    qx, qd = state["qx"], state["qd"]
+    fwd_ms, _, fclk = timed_batches(lambda i: fp4.gemm(qx, qw, out=dout, workspace=ws), args.steps, args.warmup, di)
+    bwd_ms, _, _ = timed_batches(lambda i: fp4.gemm(qd, wt, out=dxout, workspace=ws), args.steps, args.warmup, di)
+    _check(fp4)
+    flop = 2.0 * s ** 3
+    x_host, dy_host = x.pin_memory(), dy.pin_memory()
+    d_host = torch.empty(s, s, dtype=torch.bfloat16).pin_memory()
+    dx_host = torch.empty(s, s, dtype=torch.bfloat16).pin_memory()
+    xs_, dys_ = torch.empty_like(xd), torch.empty_like(dyd)
+    e2e_ms = _e2e(lambda i: step(i, xs_, dys_), [x_host, dy_host], [xs_, dys_], [d_host, dx_host], [dout, dxout],
+                  steps, args.warmup)
+    _check(fp4)
+    rec = {"value": 2 * flop / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms,
+           "steps_per_batch": steps, "batches": len(batches), "timing": "median over batches",
+           "config": {"workload": f"training-recipe step M=N=K={s}: 16x16-block NVFP4 W (and W^T) quantized once, "
+                                  "X and dY (bf16 N(0,1)) quantized every step, forward X W^T and backward dY W, "
+                                  "bf16 out", "S": s,
+                      "step": "amax + quantize X, amax + quantize dY, forward GEMM, backward GEMM (6 launches)",
+                      "l2": "X, dY (512 MiB each) and the quantized W (144 MiB) exceed the L2"},
+           "roofline": _tensor_roofline("fp4_gemm_kernel<256, nvfp4, 1 acc, CTA pair> (forward)", flop, fwd_ms, peaks,
+                                        f"train_gemm_{s}", {"gemm_clocks": fclk,
+                                                            "backward_TFLOP/s": flop / (bwd_ms * 1e-3) / 1e12,
+                                                            "backward_ms": bwd_ms}),
+           "e2e": {"value": 2 * flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                   "h2d_bytes_per_step": 2 * s * s * 2, "d2h_bytes_per_step": 2 * s * s * 2},
+           "gpu_launches_per_step": 6, "clocks": clk}
+    if cpu:
+        import oracle
+        rows = 2
+        xb = workloads.bf16_bits(x)
+        g = oracle.global_scale(oracle.amax(xb))
+        ow = oracle.quantize(w.numpy(), oracle.NVFP4, 256)
+        w_hat = oracle.dequantize(ow["codes"], ow["scales"], ow["g"])
+        del ow
+        v, cores, reps = _oracle_rows_gemm_rate(np.ascontiguousarray(xb[:rows]), oracle.NVFP4, 16, w_hat, g)
+        rec["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{reps} x (quantize {rows} rows of X with the tensor's g, FP64 product "
+                                         f"with the {s} x {s} dequantized 2-D-quantized weights)"}
+        del w_hat
+    del qw, wt, ws, dout, dxout, xd, dyd, state, xs_, dys_
+    torch.cuda.empty_cache()
+    return rec
+
+
+def measure_moe(args, dev, peaks, cpu: bool) -> dict:
+    """MXFP4 grouped MoE GEMM: 32 experts, 4096 tokens top-4 (16384 rows), K=2880, N=5760;
+    the activations are quantized (grouped layout) every step; BF16 out."""
     import block_scaled_fp4_04_b200 as fp4
     a, w, offsets, _ = workloads.moe_inputs(device="cpu")
     E, N, K = w.shape
     rows = a.shape[0]
-    a = a.to(dev)
+    ad = a.to(dev)
     wq = [fp4.quantize(w[e].to(dev), fp4.MXFP4, 32) for e in range(E)]
     B = torch.stack([q.codes for q in wq])
     sB = torch.cat([q.scales for q in wq])
@@ -440,9 +618,9 @@ def run_moe(args, dev):
     P = lambda t: t.data_ptr()
     sp = torch.cuda.current_stream().cuda_stream
 
-    def quant(i):
-        if L.fp4_quantize_grouped(P(a), rows, K, fp4.BF16, fp4.MXFP4, E, P(off), P(codes), P(scales), None, None,
-                                  None, 0, sp):
+    def quant(i, src=None):
+        if L.fp4_quantize_grouped(P(src if src is not None else ad), rows, K, fp4.BF16, fp4.MXFP4, E, P(off), P(codes),
+                                  P(scales), None, None, None, 0, sp):
             raise RuntimeError(fp4.fp4_last_error())
 
     def gemm(i):
@@ -450,124 +628,139 @@ def run_moe(args, dev):
                               fp4.BF16, None, 0, sp):
             raise RuntimeError(fp4.fp4_last_error())
 
-    step_ms = _events_ms(lambda i: (quant(i), gemm(i)), args.steps, args.warmup)
-    gemm_ms = _events_ms(gemm, args.steps, args.warmup)
-    quant_ms = _events_ms(quant, args.steps, args.warmup)
+    di = dev.index or 0
+    step_ms, batches, clk = timed_batches(lambda i: (quant(i), gemm(i)), args.steps, args.warmup, di)
+    gemm_ms, _, gclk = timed_batches(gemm, args.steps, args.warmup, di)
+    quant_ms, _, _ = timed_batches(quant, args.steps, args.warmup, di)
     _check(fp4)
     flop = 2.0 * rows * N * K
-    gemm_bytes = E * N * K // 2 + sB.numel() + rows * K // 2 + scales.numel() + rows * N * 2
+    gemm_bytes = E * N * K // 2 + sB.numel() + rows * K // 2 + rows * (K // 32) + rows * N * 2
     quant_bytes = rows * K * 2 + rows * K // 2 + rows * K // 32
-    hbm, bf16, bf16_s, src = load_peaks()
-    peak = bf16 * FP4_PER_BF16
-    t_roof = max(flop / (peak * 1e12), gemm_bytes / (hbm * 1e9)) * 1e3
-    gemm_tf = flop / (gemm_ms * 1e-3) / 1e12
-    return _line("MXFP4 grouped MoE GEMM: 32 experts, 4096 tokens top-4 (16384 rows), K=2880, N=5760, bf16 out",
-                 flop / (step_ms * 1e-3) / 1e12, "TFLOP/s", step_ms, args, {
-                     "dtype": "mxfp4 x mxfp4 -> fp32 accumulate, bf16 out",
-                     "roofline": {"bound": "tensor" if flop / peak > gemm_bytes / hbm * 1e-3 else "hbm",
-                                  "kernel": "fp4_gemm_kernel<256, mxfp4, 1, CTA pair> (grouped)",
-                                  "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
-                                  "frac": t_roof / gemm_ms,
-                                  "frac_definition": "roofline time (slower of tensor and HBM) / measured time",
-                                  "hbm_GB/s": gemm_bytes / (gemm_ms * 1e-3) / 1e9, "algorithmic_bytes": gemm_bytes,
-                                  "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g}; {src} hbm_gbs",
-                                  "launch_ms": gemm_ms, "traffic": None},
-                     "quantize": {"ms": quant_ms, "GB/s": quant_bytes / (quant_ms * 1e-3) / 1e9,
-                                  "frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / hbm},
-                     "gpu_launches": 2 * args.steps})
+    t_roof_ms = max(flop / (peaks["fp4"] * 1e12), gemm_bytes / (peaks["hbm"] * 1e9)) * 1e3
+    a_host = a.pin_memory()
+    d_host = torch.empty(rows, N, dtype=torch.bfloat16).pin_memory()
+    a_stage = torch.empty_like(ad)
+    e2e_ms = _e2e(lambda i: (quant(i, a_stage), gemm(i)), [a_host], [a_stage], [d_host], [D], args.steps, args.warmup)
+    _check(fp4)
+    achieved = flop / (gemm_ms * 1e-3) / 1e12
+    rec = {"value": flop / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms,
+           "steps_per_batch": args.steps, "batches": len(batches), "timing": "median over batches",
+           "config": {"workload": "MXFP4 grouped MoE GEMM: 32 experts, 4096 tokens routed top-4 by uniform gates "
+                                  "(16384 rows), K=2880, N=5760 per expert, bf16 activations quantized every step, "
+                                  "bf16 out",
+                      "step": "grouped MXFP4 quantize of the activations + grouped GEMM (2 launches)",
+                      "l2": "expert weights (265 MiB) exceed the L2"},
+           "roofline": {"bound": "tensor" if flop / peaks["fp4"] * 1e-9 > gemm_bytes / peaks["hbm"] else "hbm",
+                        "kernel": "fp4_gemm_kernel<256, mxfp4, 1 acc, CTA pair> (grouped)",
+                        "achieved": achieved, "peak": peaks["fp4"], "unit": "TFLOP/s",
+                        "frac": t_roof_ms / gemm_ms,
+                        "frac_definition": "roofline time (slower of tensor and HBM) / measured kernel time",
+                        "t_roof_ms": t_roof_ms, "launch_ms": gemm_ms, "algorithmic_bytes": gemm_bytes,
+                        "hbm_GB/s": gemm_bytes / (gemm_ms * 1e-3) / 1e9, "peak_source": peaks["fp4_source"] +
+                        "; hbm " + peaks["hbm_source"], "traffic": traffic_for("moe_gemm"), "gemm_clocks": gclk},
+           "quantize": {"ms": quant_ms, "GB/s": quant_bytes / (quant_ms * 1e-3) / 1e9,
+                        "frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / peaks["hbm"],
+                        "traffic": traffic_for("moe_quantize")},
+           "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                   "h2d_bytes_per_step": rows * K * 2, "d2h_bytes_per_step": rows * N * 2},
+           "gpu_launches_per_step": 2, "clocks": clk}
+    if cpu:
+        import oracle
+        ab = workloads.bf16_bits(a)
+        e = 0
+        lo = int(offsets[e])
+        ow = oracle.quantize(w[e].numpy(), oracle.MXFP4, 32)
+        w_hat = oracle.dequantize(ow["codes"], ow["scales"], ow["g"], oracle.MXFP4)
+        v, cores, reps = _oracle_rows_gemm_rate(np.ascontiguousarray(ab[lo:lo + 32]), oracle.MXFP4, 32, w_hat)
+        rec["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{reps} x (MXFP4-quantize 32 rows of expert 0's activations, FP64 product "
+                                         "with its 5760 x 2880 dequantized weights)"}
+    del B, sB, codes, scales, D, ad, a_stage
+    torch.cuda.empty_cache()
+    return rec
 
 
-def run_train(args, dev):
-    """Training-recipe sweep: W quantized once with 16x16 blocks (W and W^T); per step X and
-    dY quantized (16-blocks), forward D = X W^T and backward dX = dY W."""
+def measure_quantize(args, dev, peaks, cpu: bool) -> dict:
+    """The quantize kernels alone (GB/s of algorithmic bytes; NVFP4 reads x twice: the tensor
+    amax, then the encode)."""
     import block_scaled_fp4_04_b200 as fp4
-    hbm, bf16, bf16_s, src = load_peaks()
-    peak = bf16 * FP4_PER_BF16
-    out = []
-    for s in (1024, 2048, 4096, 8192, 16384):
-        x, w, dy = workloads.train_inputs(s, device="cpu")
-        per_copy = 2 * s * s * 2
-        ncopy = _copies(per_copy) if s <= 2048 else 1
-        xs = [x.to(dev) for _ in range(ncopy)]
-        dys = [dy.to(dev) for _ in range(ncopy)]
-        qw = fp4.quantize(w.to(dev), fp4.NVFP4, 256)
-        wt = fp4.transposed(qw)
-        ws = fp4.Workspace(dev)
-        dout = torch.empty(s, s, dtype=torch.bfloat16, device=dev)
-        dxout = torch.empty(s, s, dtype=torch.bfloat16, device=dev)
-        state = {}
-
-        def step(i):
-            qx = fp4.quantize(xs[i % ncopy], fp4.NVFP4, 16, workspace=ws)
-            qd = fp4.quantize(dys[i % ncopy], fp4.NVFP4, 16, workspace=ws)
-            fp4.gemm(qx, qw, out=dout, workspace=ws)
-            fp4.gemm(qd, wt, out=dxout, workspace=ws)
-            state["qx"], state["qd"] = qx, qd
-
-        step_ms = _events_ms(step, max(3, args.steps // 4), args.warmup)
-        qx, qd = state["qx"], state["qd"]
-        fwd_ms = _events_ms(lambda i: fp4.gemm(qx, qw, out=dout, workspace=ws), args.steps, args.warmup)
-        bwd_ms = _events_ms(lambda i: fp4.gemm(qd, wt, out=dxout, workspace=ws), args.steps, args.warmup)
-        _check(fp4)
-        flop = 2.0 * s * s * s
-        out.append({"S": s, "step_ms": step_ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
-                    "fwd_TFLOP/s": flop / (fwd_ms * 1e-3) / 1e12, "bwd_TFLOP/s": flop / (bwd_ms * 1e-3) / 1e12,
-                    "fwd_frac": flop / (fwd_ms * 1e-3) / 1e12 / peak,
-                    "step_TFLOP/s": 2 * flop / (step_ms * 1e-3) / 1e12,
-                    "l2": f"{ncopy} rotating copies of X, dY" if ncopy > 1 else "inputs larger than L2"})
-        del xs, dys, qw, wt, ws, dout, dxout, state
-        torch.cuda.empty_cache()
-    big = out[-1]
-    return _line("training-recipe sweep M=N=K in {1024..16384}: 2-D NVFP4 W (and W^T) once, X and dY quantized "
-                 "per step, forward X W^T and backward dY W, bf16 out", big["step_TFLOP/s"], "TFLOP/s",
-                 big["step_ms"], args, {
-                     "dtype": "nvfp4 x nvfp4 -> fp32 accumulate, bf16 out",
-                     "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, nvfp4, 1, CTA pair> at S=16384",
-                                  "achieved": big["fwd_TFLOP/s"], "peak": peak, "unit": "TFLOP/s",
-                                  "frac": big["fwd_frac"], "traffic": None,
-                                  "peak_source": f"{src} bf16_tflops x {FP4_PER_BF16:g}"},
-                     "sweep": out, "gpu_launches": None})
-
-
-def run_quantize(args, dev):
-    """Quantize kernels alone: GB/s of algorithmic bytes (NVFP4 reads x twice: amax, encode)."""
-    import block_scaled_fp4_04_b200 as fp4
-    hbm, bf16, bf16_s, src = load_peaks()
-    rows_out = []
     cases = [
-        ("moe activations bf16 [16384, 2880] -> MXFP4", lambda: workloads.moe_inputs(device="cpu")[0], fp4.MXFP4, 32),
-        ("train X bf16 [16384, 16384] -> NVFP4", lambda: workloads.train_inputs(16384, device="cpu")[0], fp4.NVFP4, 16),
-        ("decode W fp32 [28672, 8192] -> NVFP4", lambda: workloads.decode_inputs(device="cpu")[1], fp4.NVFP4, 16),
-        ("2-D W fp32 [16384, 16384] -> NVFP4 W and W^T", lambda: workloads.train_inputs(16384, device="cpu")[1],
-         fp4.NVFP4, 256),
+        ("moe_quantize", "MoE activations bf16 [16384, 2880] -> MXFP4",
+         lambda: workloads.moe_inputs(device="cpu", n=32)[0], fp4.MXFP4, 32),
+        ("quantize_train_x", "train X bf16 [16384, 16384] -> NVFP4 (amax + encode)",
+         lambda: workloads.train_inputs(16384, device="cpu")[0], fp4.NVFP4, 16),
+        ("quantize_decode_w", "decode W fp32 [28672, 8192] -> NVFP4 (amax + encode)",
+         lambda: workloads.decode_inputs(device="cpu")[1], fp4.NVFP4, 16),
+        ("quantize_2d_w", "2-D W fp32 [16384, 16384] -> NVFP4 W and W^T (amax + encode)",
+         lambda: workloads.train_inputs(16384, device="cpu")[1], fp4.NVFP4, 256),
     ]
-    for name, make, fmt, blk in cases:
-        x = make().to(dev)
+    out = []
+    di = dev.index or 0
+    train = {}
+
+    def train_tensor(j):
+        if not train:
+            x, w, _ = workloads.train_inputs(16384, device="cpu")
+            train.update(x=x, w=w)
+        return train["x" if j == 0 else "w"]
+
+    cases[1] = cases[1][:2] + (lambda: train_tensor(0),) + cases[1][3:]
+    cases[3] = cases[3][:2] + (lambda: train_tensor(1),) + cases[3][3:]
+    for key, name, make, fmt, blk in cases:
+        xh = make()
+        x = xh.to(dev)
         rows, cols = x.shape
         esz = x.element_size()
         ws = fp4.Workspace(dev)
         codes = rows * cols // 2
         sc = fp4.fp4_scales_bytes(rows, cols, fmt)
         if blk == 256:
-            nbytes = 2 * rows * cols * esz + 2 * (codes + sc)   # amax read + encode read; W and W^T
+            nbytes = 2 * rows * cols * esz + 2 * (codes + sc)
         elif fmt == fp4.NVFP4:
             nbytes = 2 * rows * cols * esz + codes + sc
         else:
             nbytes = rows * cols * esz + codes + sc
-        ms = _events_ms(lambda i: fp4.quantize(x, fmt, blk, workspace=ws), max(3, args.steps // 4), args.warmup)
+        ms, batches, clk = timed_batches(lambda i: fp4.quantize(x, fmt, blk, workspace=ws), max(3, args.steps // 4),
+                                         args.warmup, di, min_s=0.25)
         _check(fp4)
         gbs = nbytes / (ms * 1e-3) / 1e9
-        rows_out.append({"case": name, "ms": ms, "GB/s": gbs, "frac": gbs / hbm, "bytes": nbytes})
-        del x, ws
+        rec = {"case": name, "ms": ms, "GB/s": gbs, "bytes": nbytes,
+               "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                            "frac": gbs / peaks["hbm"], "peak_source": peaks["hbm_source"],
+                            "traffic": traffic_for(key)}, "clocks": clk}
+        if cpu and key in ("moe_quantize", "quantize_train_x"):
+            import oracle
+            xb = workloads.bf16_bits(xh) if xh.dtype == torch.bfloat16 else xh.numpy()
+            sample = np.ascontiguousarray(xb[:256])
+            t0 = time.perf_counter()
+            reps = 0
+            while time.perf_counter() - t0 < 2.0 and reps < 50:
+                oracle.quantize(sample, fmt, blk)
+                reps += 1
+            dt = time.perf_counter() - t0
+            per = sample.shape[0] * cols * esz * (2 if fmt == fp4.NVFP4 else 1) + sample.shape[0] * cols // 2
+            rec["cpu_baseline"] = {"value": per * reps / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+                                   "kind": "oracle", "sample": f"{reps} x 256 rows of the same tensor"}
+        out.append(rec)
+        del x, ws, xh
         torch.cuda.empty_cache()
-    best = rows_out[0]
-    return _line("quantize kernels alone (MoE activations, train X, decode W, 2-D W)", best["GB/s"], "GB/s",
-                 best["ms"], args, {
-                     "dtype": "bf16/fp32 in -> nvfp4/mxfp4 codes + scales",
-                     "roofline": {"bound": "hbm", "kernel": "quantize (first case)", "achieved": best["GB/s"],
-                                  "peak": hbm, "unit": "GB/s", "frac": best["frac"], "traffic": None,
-                                  "peak_source": f"{src} hbm_gbs"},
-                     "cases": rows_out, "gpu_launches": None})
+    return {"cases": out}
+
+
+def load_peak_table(dev) -> dict:
+    hbm, bf16, bf16_s, src = load_peaks()
+    pk = {"hbm": hbm, "hbm_source": f"{src} hbm_gbs (MEASURED_PEAKS.json)" if src == "measured" else src,
+          "fp4": bf16 * FP4_PER_BF16,
+          "fp4_source": f"{src} bf16_tflops {bf16:g} x {FP4_PER_BF16:g} (nominal FP4/BF16 dense ratio)"}
+    try:
+        pk["mma_loop_record"] = mma_peak(dev)
+        pk["mma_loop"] = pk["mma_loop_record"]["TFLOP/s"]
+    except Exception as e:  # the probe is context; its failure does not stop the bench
+        pk["mma_loop_record"] = {"error": str(e)[:200]}
+    return pk
+
+
+MEASURES = {"prefill": measure_prefill, "train": measure_train, "moe": measure_moe, "quantize": measure_quantize}
 
 
 def cpu_baseline_decode(budget_s: float = 12.0):
@@ -582,30 +775,19 @@ def cpu_baseline_decode(budget_s: float = 12.0):
     wq = oracle.quantize(w[:rows].numpy(), oracle.NVFP4, 16, g_in=g_w)
     xb = workloads.bf16_bits(x)
     t0 = time.perf_counter()
-    done = 0
     reps = 0
     while True:
         xq = oracle.quantize(xb, oracle.NVFP4, 16)
         xh = oracle.dequantize(xq["codes"], xq["scales"], xq["g"])
         wh = oracle.dequantize(wq["codes"], wq["scales"], wq["g"])
         oracle.gemm_reference(xh, wh)
-        done += rows
         reps += 1
         if time.perf_counter() - t0 > budget_s or reps >= 64:
             break
     dt = time.perf_counter() - t0
     _, _, per_step = decode_bytes(m, rows, k)
     gbs = per_step * reps / dt / 1e9
-    return gbs, _cores(), f"{reps} x (quantize X 16x8192 + {rows} weight rows of 28672) in {dt:.1f} s"
-
-
-def _cores() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        th = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max([1] + th)
-    except Exception:
-        return 1
+    return gbs, oracle.num_threads(), f"{reps} x (quantize X 16x8192 + {rows} weight rows of 28672) in {dt:.1f} s"
 
 
 def run_reference(args, dist: Dist):
@@ -646,7 +828,8 @@ def run_reference(args, dist: Dist):
         "data": "synthetic (seeded, same recipe as the GPU arm)",
         "config": {"workload": "decode-shaped NVFP4 GEMM M=16 N=28672 K=8192 (bounded sample per step)",
                    "sample": sample},
-        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": _cores(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -654,15 +837,21 @@ def run_reference(args, dist: Dist):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "train", "quantize", "all"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "train", "quantize"],
+                    help="decode: the headline line, with the other configurations as sub-records; any other "
+                         "value prints that configuration's record alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other configurations' sub-records")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")
     dist = Dist()
+    if args.gpus != dist.world:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} ranks (WORLD_SIZE is {dist.world}): launch with "
+                         f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus}")
     if args.impl == "reference":
         if dist.rank == 0:
             print(json.dumps(run_reference(args, dist)))
@@ -670,21 +859,28 @@ def main():
     torch.cuda.set_device(dist.local)
     dev = torch.device("cuda", dist.local)
     dist.init("nccl")
+    cpu = not args.no_cpu_baseline
     try:
         if args.workload != "decode":
             if dist.world > 1:
-                raise SystemExit("the additional workloads run on one GPU")
-            names = ["prefill", "moe", "train", "quantize"] if args.workload == "all" else [args.workload]
-            for name in names:
-                print(json.dumps({"prefill": run_prefill, "moe": run_moe, "train": run_train,
-                                  "quantize": run_quantize}[name](args, dev)), flush=True)
+                raise SystemExit("the other configurations run on one GPU")
+            peaks = load_peak_table(dev)
+            rec = MEASURES[args.workload](args, dev, peaks, cpu)
+            rec.update({"metric": METRIC, "n_gpus": 1, "peaks": {k: v for k, v in peaks.items() if k != "mma_loop"}})
+            print(json.dumps(rec), flush=True)
             return
         res = run_decode(args, dist, dev)
         if dist.rank == 0:
-            if dist.world == 1 and not args.no_cpu_baseline:
+            if dist.world == 1 and cpu:
                 v, cores, sample = cpu_baseline_decode()
                 res["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle",
                                        "sample": sample}
+            if dist.world == 1 and not args.no_extra:
+                peaks = load_peak_table(dev)
+                res["peaks"] = {k: v for k, v in peaks.items() if k != "mma_loop"}
+                res["workloads"] = {}
+                for name, fn in MEASURES.items():
+                    res["workloads"][name] = fn(args, dev, peaks, cpu)
             print(json.dumps(res))
     finally:
         dist.close()

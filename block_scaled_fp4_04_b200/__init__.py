@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
                 "fp4_gemm_grouped": (I32, [I32, I32, P, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_get_status": (I32, [P]),
                 "fp4_debug_encode": (I32, [P, I64, I32, P, P]),
+                "fp4_debug_stall_next_decode": (I32, [I32]),
+                "fp4_mma_peak": (I32, [I32, I32, P, P]),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(L, name)
@@ -236,6 +238,14 @@ def fp4_gemm_grouped(fmt, num_groups, offsets, A, sA, gA, B, sB, gB, total_rows,
 def fp4_get_status(stream=None) -> int:
     """Synchronizes the stream and returns (and clears) the latched device status."""
     return int(lib().fp4_get_status(_s(stream)))
+
+
+def fp4_mma_peak(iters: int, grid: int, cycles, stream=None):
+    _check(lib().fp4_mma_peak(iters, grid, _p(cycles), _s(stream)))
+
+
+def fp4_debug_stall_next_decode(cta: int):
+    _check(lib().fp4_debug_stall_next_decode(cta))
 
 
 def fp4_debug_encode(inp, n, which, out, stream=None):

@@ -68,6 +68,10 @@ static fp4_status device_state(unsigned** status) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Test hook (fp4_debug_stall_next_decode): the CTA whose amax share the next fused decode
+// launch of this thread leaves unpublished, plus one (0: none).
+static thread_local int g_stall_next_decode = 0;
+
 }  // namespace fp4
 
 using namespace fp4;
@@ -327,6 +331,13 @@ fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, c
   g.q_codes = Dcodes;
   g.q_scales = Dscales;
   g.q_g = gD;
+  if (Dcodes && (M % 128 != 0 || (N / 16) % 4 != 0)) {
+    // the kernel writes the scale bytes of real rows and blocks; the layout's pad bytes
+    // (rows up to a multiple of 128, block columns up to a multiple of 4) must read as 0
+    const cudaError_t e =
+        cudaMemsetAsync(Dscales, 0, fp4_scales_bytes(M, N, FP4_NVFP4), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "zero-filling the scale pads");
+  }
   return gemm_common(g, fmt, out_dtype, stream);
 }
 
@@ -375,6 +386,8 @@ fp4_status fp4_gemm_bf16a(const void* X, const uint8_t* B, const uint8_t* sB, co
     q.ws = static_cast<uint8_t*>(workspace) + qws;
     q.ws_bytes = workspace_bytes - qws;
     q.weights_ready = (flags & FP4_GEMM_WEIGHTS_READY) ? 1 : 0;
+    q.stall_plus1 = g_stall_next_decode;
+    g_stall_next_decode = 0;
     const char* why = nullptr;
     cudaError_t err = cudaSuccess;
     const int rc = launch_decode(q, status, static_cast<cudaStream_t>(stream), &why, &err);
@@ -492,6 +505,22 @@ fp4_status fp4_get_status(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "status clear");
   if (v & kStatusTimeout) return fail(FP4_ERR_TIMEOUT, "a device-side wait timed out");
   if (v & kStatusNonFinite) return fail(FP4_ERR_NONFINITE, "non-finite input element");
+  return FP4_OK;
+}
+
+fp4_status fp4_mma_peak(int iters, int grid, unsigned long long* cycles, void* stream) {
+  if (!cycles || iters <= 0 || iters > (1 << 24) || grid <= 0 || grid > 4 * num_sms())
+    return fail(FP4_ERR_INVALID_ARG, "iters in 1..2^24, grid in 1..4 x SMs, cycles non-null");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  const cudaError_t e = launch_mma_peak(iters, grid, cycles, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "MMA peak launch");
+}
+
+fp4_status fp4_debug_stall_next_decode(int cta) {
+  if (cta < 0) return fail(FP4_ERR_INVALID_ARG, "cta must be >= 0");
+  g_stall_next_decode = cta + 1;
   return FP4_OK;
 }
 

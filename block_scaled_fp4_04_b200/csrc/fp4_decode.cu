@@ -56,6 +56,8 @@ struct DecodeArgs {
   unsigned* status;
   const float* bias;      // [N] added to every output row after the scale, or null
   int act;                // 0: none, 1: ReLU
+  int stall_plus1;        // test hook for the bounded waits: CTA stall_plus1 - 1 does not
+                          // publish its share of the amax (0: every CTA publishes)
 };
 
 // K steps of one segment at most (the activations' scale factors for a segment take 16
@@ -493,7 +495,8 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         const uint32_t gen = *reinterpret_cast<volatile unsigned*>(p.gbar) + 1u;
         s_red[8] = gen;
         const uint64_t word = (static_cast<uint64_t>(gen) << 32) | cm;
-        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(slots + blockIdx.x * 16), "l"(word) : "memory");
+        if (static_cast<int>(blockIdx.x) + 1 != p.stall_plus1)
+          asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(slots + blockIdx.x * 16), "l"(word) : "memory");
       }
       named_sync(3, 256);
       const uint32_t gen = s_red[8];
@@ -900,6 +903,7 @@ int launch_decode(const DecodeProblem& q, unsigned* status, cudaStream_t st, con
   a.status = status;
   a.bias = q.bias;
   a.act = q.act;
+  a.stall_plus1 = q.stall_plus1;
   const int grid = pl.nseg * pl.ctas_per_seg;
   cudaError_t e;
   if (q.X) e = BN == 16 ? run_decode<16, true>(tw, tx, a, grid, st) : run_decode<32, true>(tw, tx, a, grid, st);

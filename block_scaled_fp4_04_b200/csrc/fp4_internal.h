@@ -47,6 +47,7 @@ cudaError_t launch_set_value(float* p, float v, cudaStream_t st);
 // g = amax / (6 * 448), 1 when amax is 0; a non-finite amax latches kStatusNonFinite.
 cudaError_t launch_global_scale(const float* amax, float* g, unsigned* status, cudaStream_t st);
 cudaError_t launch_debug_encode(const float* in, int64_t n, int which, uint8_t* out, cudaStream_t st);
+cudaError_t launch_mma_peak(int iters, int grid, unsigned long long* cycles, unsigned* status, cudaStream_t st);
 
 // GEMM problem as the host API sees it (see fp4.h for the meaning of each field).
 struct GemmProblem {
@@ -97,6 +98,7 @@ struct DecodeProblem {
   int weights_ready;
   const float* bias;  // [N] or null
   int act;            // 0 none, 1 ReLU
+  int stall_plus1;    // test hook: CTA stall_plus1 - 1 never publishes its amax share (0: none)
 };
 bool decode_eligible(int64_t M, int64_t N, int64_t K);
 size_t decode_workspace_bytes(int64_t M, int64_t N);

@@ -218,7 +218,8 @@ fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev,
  *           codes [M, N/2], scales fp4_scales_bytes(M, N, FP4_NVFP4) in the swizzled
  *           layout, quantized exactly as fp4_quantize would quantize the FP32 t with
  *           global_in = gD_dev (the caller's global scale: t's amax is not known until
- *           the whole product is, so it cannot be computed here).  The result can feed
+ *           the whole product is, so it cannot be computed here).  The layout's pad
+ *           bytes are written as 0, as fp4_quantize writes them.  The result can feed
  *           the next fp4_gemm as its A operand directly.  Needs N % 32 == 0.
  *   bias_dev [N] FP32 or NULL; act FP4_ACT_NONE or FP4_ACT_RELU.
  * workspace: fp4_gemm_epilogue_workspace_size(M, N, K, fmt, Dcodes_dev != NULL) bytes,
@@ -291,6 +292,23 @@ fp4_status fp4_gemm_grouped(fp4_fmt fmt, int num_groups, const int32_t* offsets_
  * (after synchronizing `stream`).  Returns FP4_OK, FP4_ERR_NONFINITE or FP4_ERR_TIMEOUT
  * (the first error latched), or FP4_ERR_CUDA if the synchronization failed. */
 fp4_status fp4_get_status(void* stream);
+
+/* Measured peak of the block-scaled tensor-core MMA ("NVIDIA FP4" article, hardware table:
+ * 9 PFLOP/s dense FP4 on B200 is the vendor's figure; this measures what the tensor pipe
+ * sustains here).  grid CTAs (one per SM) each issue iters x 4 back-to-back
+ * tcgen05.mma.kind::mxf4nvf4 of M = 128, N = 256, K = 64 from shared memory into TMEM,
+ * with no loads and no epilogue, and write the loop's clock64 cycles to cycles_dev[cta].
+ * Each CTA does 2 * 128 * 256 * 64 * 4 * iters FLOP; time the launch with events on
+ * `stream` for FLOP/s.  iters <= 2^24. */
+fp4_status fp4_mma_peak(int iters, int grid, unsigned long long* cycles_dev, void* stream);
+
+/* Test hook for the device-side bounded waits (tests only): the next fp4_gemm_bf16a call
+ * of this thread that takes the single-launch decode path runs with CTA `cta` never
+ * publishing its share of the activations' tensor amax.  Every CTA's bounded wait for
+ * that share then runs out (after about 2 s), the call latches FP4_ERR_TIMEOUT, every
+ * CTA releases its resources and returns, and the outputs are unspecified.  Zero-fill
+ * the workspace before its next use.  A cta beyond the grid has no effect. */
+fp4_status fp4_debug_stall_next_decode(int cta);
 
 /* Encoder check entry point (tests): out_dev[i] = the code the device encoders give
  * in_dev[i] (no scaling), i < n.  which = 0: E2M1 code (sign in bit 3) from the encoder

@@ -132,3 +132,15 @@ def test_reduce_amax_is_a_no_op_without_a_process_group():
     from block_scaled_fp4_04_b200 import sharded
     t = torch.tensor([2.5])
     assert sharded.reduce_amax_(t).item() == 2.5
+
+
+def test_bench_refuses_a_gpu_count_without_matching_ranks():
+    """`bench.py --gpus 2` outside torchrun would silently measure one GPU: it stops with
+    a message naming the launch command instead (before touching a GPU)."""
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"), "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode != 0
+    assert "--nproc-per-node 2" in r.stderr

@@ -298,3 +298,29 @@ def test_gemm_bf16a_full_decode_shape_sampled():
     d_ref, s = oracle.gemm_reference(dequant_oracle(ox, fp4.NVFP4), b_hat)
     got = d[:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - d_ref) <= oracle.gemm_tolerance(d_ref, s, True))
+
+
+def test_bounded_wait_runs_out_and_the_next_call_is_correct():
+    """The decode kernel's CTAs wait (bounded) for each other's share of the activations'
+    amax.  With one share never published (the test hook), every wait runs out: the call
+    latches FP4_ERR_TIMEOUT and returns; the device stays usable, and the next call on a
+    zero-filled workspace gives the oracle's result."""
+    m, n, k = 16, 2048, 4096
+    xa = random_input(m, k, 61, torch.bfloat16).cuda()
+    xb = random_input(n, k, 62, torch.float32, std=0.02, outliers=False)
+    qb = gpu_quantize(xb.cuda(), fp4.NVFP4, 16)
+    ws = torch.zeros(fp4.fp4_gemm_bf16a_workspace_size(m, n, k), dtype=torch.uint8, device="cuda")
+    fp4.fp4_debug_stall_next_decode(3)
+    xq = torch.empty(m, k // 2, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(fp4.fp4_scales_bytes(m, k, fp4.NVFP4), dtype=torch.uint8, device="cuda")
+    gx = torch.empty(1, dtype=torch.float32, device="cuda")
+    d = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    fp4.fp4_gemm_bf16a(xa, qb.codes, qb.scales, qb.g, m, n, k, d, fp4.BF16, xq, xs, gx, ws, ws.numel())
+    assert fp4.fp4_get_status() == fp4.ERR_TIMEOUT
+    assert fp4.fp4_get_status() == fp4.OK          # read and cleared
+    ws.zero_()
+    d2, qx, _ = _bf16a(xa, qb, n, k, ws=ws)
+    from fp4_testutil import assert_quant_equal
+    ox, ob = oracle_quantize(xa.cpu(), fp4.NVFP4, 16), oracle_quantize(xb, fp4.NVFP4, 16)
+    assert_quant_equal(qx, ox, "after the timeout")
+    check_gemm(d2, dequant_oracle(ox, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label="after the timeout")
