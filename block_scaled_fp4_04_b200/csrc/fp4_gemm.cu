@@ -236,14 +236,7 @@ struct Cfg {
   // is few enough registers to hold the tile while TMEM is already handed back.
   static constexpr int kEpiWarps = kSepCp ? 8 : 4;
   static constexpr int kEpiCols = BN * 4 / kEpiWarps;  // accumulator columns per epilogue thread
-  // Single-pipeline kernels also split the loads over two producer warps on different
-  // SM sub-partitions (warp 0: A and its scales; kProdBWarp: B and its scales): one
-  // thread issues a TMA copy only every ~200 cycles, so a single producer cannot keep up
-  // with a 256-deep K step of M = 256 MMAs (~540 cycles) when a stage takes five copies.
-  static constexpr int kProdBWarp = 2 + kEpiWarps;
-  static constexpr int kCopier0 = kSepCp ? kProdBWarp + 1 : 0;
-  static constexpr int kProducers = kSepCp ? 2 : 1;
-  static constexpr int kThreads = kSepCp ? 64 + 32 * kEpiWarps + 32 + 32 * kCopiers : 192 * kP;
+  static constexpr int kThreads = kSepCp ? 64 + 32 * kEpiWarps + 32 * kCopiers : 192 * kP;
   static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
@@ -443,9 +436,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
   // prologue (overlaps the tail of the previous kernel under programmatic launch)
   if (lt == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], C::kProducers);  // one arrival (with its byte count) per producer
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_landed[s], C::kProducers);
+      mbar_init(&sf_landed[s], 1);
     }
     for (int a = 0; a < ACC; ++a) {
       mbar_init(&acc_full[a], 1);
@@ -535,9 +528,9 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
                       smem_desc_sf(st + C::kABytes + C::kBBytes + C::kSFABytes + (rb * C::kAtomsKT + a) * 512));
   };
 
-  if (warp == 0 || (C::kSepCp && warp == C::kProdBWarp)) {
+  if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------------ producer(s)
+      // ------------------------------------------------------------ producer
       // swapped decode: the weights (A here) are read once -> evict first; the small
       // activations (B) are re-read by every CTA -> keep
       // otherwise both operands are re-read by other tiles -> keep (the output is stored
@@ -583,103 +576,72 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
           tma_load_2d(st + C::kABytes, &tmB, &full[st_idx], kb * 128, w.b_row, pol_b);
         }
       };
-      // scale-factor bytes of one side of a stage (B: only the row-blocks that exist)
-      auto side_sf_bytes = [&](const Work& w, int kb, bool side_a) -> uint32_t {
+      auto stage_sf_bytes = [&](const Work& w, int kb) -> uint32_t {
         const int atoms = min(C::kAtomsKT, p.sf_atoms_k - kb * C::kAtomsKT);
         const uint32_t sf_bytes = static_cast<uint32_t>(atoms) * 512u;
-        if (side_a) return sf_bytes;
         const int rb0 = w.n0 / 128;
         int nrb = 0;
 #pragma unroll
         for (int rb = 0; rb < C::kNRB; ++rb) nrb += (rb0 + rb < p.sfb_rbs) ? 1 : 0;
-        return sf_bytes * nrb;
+        return sf_bytes * (1 + nrb);
       };
+      // With an independent operand, the first ring-full of stages loads only that side,
+      // then waits for the preceding kernel, then issues the other side of those stages.
+      const bool early = p.indep != 0;
+      const bool early_a = p.indep == 1;
+      int npend = 0;
+      bool replayed = !early;
+      auto replay = [&]() {
+        wait_prior_grids();
+        Sched<BN> rs(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
+        Work rw;
+        int j = 0;
+        while (j < npend && rs.next(rw))
+          for (int kb = rw.kb0; kb < rw.kb1 && j < npend; ++kb, ++j) load_side(j, rw, kb, !early_a);
+        replayed = true;
+      };
+      if (!early) wait_prior_grids();
       Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
       Work w;
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
       bool ok = true;
-      if constexpr (C::kSepCp) {
-        // Two producers: this warp loads one side (A and its scales, or B and its scales)
-        // of every stage and arrives on the stage's barriers with that side's byte count.
-        // A side the caller marked as ready is loaded without waiting for the preceding
-        // kernel; the other producer waits for it first.
-        const bool side_a = warp == 0;
-        const bool ready = (p.indep == 1 && side_a) || (p.indep == 2 && !side_a);
-        if (!ready) wait_prior_grids();
-        while (ok && sch.next(w)) {
-          for (int kb = w.kb0; kb < w.kb1; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, s_abort)) {
-              latch_timeout(s_abort, p.status);
-              ok = false;
-              break;
+      while (ok && sch.next(w)) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort)) {
+            latch_timeout(s_abort, p.status);
+            ok = false;
+            break;
+          }
+          if constexpr (PAIR) {
+            if (leader) {  // the leader's barriers count the boxes of both CTAs
+              mbar_arrive_expect_tx(&sf_landed[stage], 2 * (C::kSFABytes + C::kSFBBytes));
+              mbar_arrive_expect_tx(&full[stage], 2 * (C::kABytes + C::kBBytes));
             }
-            if constexpr (PAIR) {
-              if (leader) {  // the leader's barriers count this side's boxes of both CTAs
-                mbar_arrive_expect_tx(&sf_landed[stage], 2 * (side_a ? C::kSFABytes : C::kSFBBytes));
-                mbar_arrive_expect_tx(&full[stage], 2 * (side_a ? C::kABytes : C::kBBytes));
-              }
-            } else {
-              mbar_arrive_expect_tx(&sf_landed[stage], side_sf_bytes(w, kb, side_a));
-              mbar_arrive_expect_tx(&full[stage], side_a ? C::kABytes : C::kBBytes);
-            }
-            load_side(stage, w, kb, side_a);
-            issued |= 1u << stage;
-            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1;
-            }
+          } else if constexpr (C::kSepCp) {
+            mbar_arrive_expect_tx(&sf_landed[stage], stage_sf_bytes(w, kb));
+            mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + stage_sf_bytes(w, kb));
+          }
+          if (!replayed) {
+            load_side(stage, w, kb, early_a);
+            if (++npend == S) replay();
+          } else {
+            load_side(stage, w, kb, true);
+            load_side(stage, w, kb, false);
+          }
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
           }
         }
-      } else {
-        // One producer for both sides.  With an independent operand, the first ring-full
-        // of stages loads only that side, then waits for the preceding kernel, then issues
-        // the other side of those stages.
-        const bool early = p.indep != 0;
-        const bool early_a = p.indep == 1;
-        int npend = 0;
-        bool replayed = !early;
-        auto replay = [&]() {
-          wait_prior_grids();
-          Sched<BN> rs(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
-          Work rw;
-          int j = 0;
-          while (j < npend && rs.next(rw))
-            for (int kb = rw.kb0; kb < rw.kb1 && j < npend; ++kb, ++j) load_side(j, rw, kb, !early_a);
-          replayed = true;
-        };
-        if (!early) wait_prior_grids();
-        while (ok && sch.next(w)) {
-          for (int kb = w.kb0; kb < w.kb1; ++kb) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, s_abort)) {
-              latch_timeout(s_abort, p.status);
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + side_sf_bytes(w, kb, true) +
-                                                    side_sf_bytes(w, kb, false));
-            if (!replayed) {
-              load_side(stage, w, kb, early_a);
-              if (++npend == S) replay();
-            } else {
-              load_side(stage, w, kb, true);
-              load_side(stage, w, kb, false);
-            }
-            issued |= 1u << stage;
-            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1;
-            }
-          }
-        }
-        if (ok && !replayed) replay();
       }
+      if (ok && !replayed) replay();
       // let every issued copy land before the CTA's shared memory goes away (a pair's
-      // leader waits for both CTAs' boxes: they complete on its barriers).  With two
-      // producers a stage whose other side was never issued does not complete; its wait
-      // runs out, long after this side's copies have landed.
+      // leader waits for both CTAs' boxes: they complete on its barriers)
       if (*s_abort && leader) {
         for (int s = 0; s < S; ++s)
           if (issued & (1u << s)) {
@@ -773,8 +735,8 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
-  } else if (C::kSepCp && warp >= C::kCopier0) {
-    const int cw = warp - C::kCopier0;  // 0: A's atoms; 1 + rb: B's row-block rb
+  } else if (C::kSepCp && warp >= 2 + C::kEpiWarps) {
+    const int cw = warp - 2 - C::kEpiWarps;  // 0: A's atoms; 1 + rb: B's row-block rb
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ scale-factor copier
       // Stage n's atoms go to TMEM slot n % kSFSlots once they have landed and the
