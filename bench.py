@@ -492,9 +492,22 @@ def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
                          P(ws), wn, 0, sp):
             raise RuntimeError(fp4.fp4_last_error())
 
+    # the GEMM with the epilogue of the next row: + bias, ReLU, and an NVFP4 copy of the result
+    bias = torch.randn(n, device=dev)
+    q_codes = torch.empty(m, n // 2, dtype=torch.uint8, device=dev)
+    q_scales = torch.empty(fp4.fp4_scales_bytes(m, n, fp4.NVFP4), dtype=torch.uint8, device=dev)
+    q_g = torch.tensor([0.05], dtype=torch.float32, device=dev)
+
+    def gemm_epi(i):
+        q = wq[i % copies]
+        if L.fp4_gemm_epilogue(fp4.NVFP4, P(xc), P(xs), P(xg), P(q.codes), P(q.scales), P(q.g), m, n, k, P(bias),
+                               fp4.ACT_RELU, P(d), fp4.BF16, P(q_codes), P(q_scales), P(q_g), P(ws), wn, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
     di = dev.index or 0
     step_ms, batches, clk = timed_batches(step, args.steps, args.warmup, di)
     gemm_ms, _, gclk = timed_batches(gemm, args.steps, args.warmup, di)
+    epi_ms, _, eclk = timed_batches(gemm_epi, args.steps, args.warmup, di)
     _check(fp4)
     flop = 2.0 * m * n * k
     x_host = x.pin_memory()
@@ -513,6 +526,10 @@ def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
                                         "prefill_gemm", {"gemm_clocks": gclk}),
            "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                    "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2},
+           "epilogue_gemm": {"what": "fp4_gemm_epilogue: + bias, ReLU, BF16 out and an NVFP4 copy of the result",
+                             "ms": epi_ms, "TFLOP/s": flop / (epi_ms * 1e-3) / 1e12,
+                             "frac": flop / (epi_ms * 1e-3) / 1e12 / peaks["fp4"], "clocks": eclk,
+                             "traffic": traffic_for("prefill_gemm_epilogue")},
            "gpu_launches_per_step": 3, "clocks": clk}
     if cpu:
         import oracle
@@ -525,7 +542,7 @@ def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
         rec["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                "sample": f"{reps} x (quantize {rows} rows of X with the tensor's g, FP64 product "
                                          f"with the 8192 x 8192 dequantized weights)"}
-    del wq, xd, xc, xs, ws, d, x_stage
+    del wq, xd, xc, xs, ws, d, x_stage, q_codes, q_scales, bias
     torch.cuda.empty_cache()
     return rec
 
@@ -744,7 +761,64 @@ def measure_quantize(args, dev, peaks, cpu: bool) -> dict:
         out.append(rec)
         del x, ws, xh
         torch.cuda.empty_cache()
+    out.extend(measure_quantize_variants(args, dev, peaks, train_tensor))
     return {"cases": out}
+
+
+def measure_quantize_variants(args, dev, peaks, train_tensor) -> list:
+    """The quantizer variants of the next rows, on the training tensors: stochastic rounding
+    (one 4-byte random word per element read as well), the 16-point Hadamard transform
+    before quantizing (the amax pass transforms too), and MXFP4 with the rounded-down
+    scale."""
+    import block_scaled_fp4_04_b200 as fp4
+    di = dev.index or 0
+    s = 16384
+    x = train_tensor(0).to(dev)
+    ws = torch.zeros(fp4.fp4_quantize_workspace_size(), dtype=torch.uint8, device=dev)
+    codes = torch.empty(s, s // 2, dtype=torch.uint8, device=dev)
+    sc16 = torch.empty(fp4.fp4_scales_bytes(s, s, fp4.NVFP4), dtype=torch.uint8, device=dev)
+    sc32 = torch.empty(fp4.fp4_scales_bytes(s, s, fp4.MXFP4), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    rbits = torch.randint(-2 ** 31, 2 ** 31 - 1, (s, s), dtype=torch.int32, device=dev, generator=gen)
+    L = fp4.lib()
+    P = lambda t: t.data_ptr()
+    sp = torch.cuda.current_stream().cuda_stream
+    n = s * s
+
+    def sr(i):
+        if L.fp4_quantize_sr(P(x), s, s, fp4.BF16, P(rbits), P(codes), P(sc16), P(g), None, P(ws), ws.numel(), sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    def rht(i):
+        if L.fp4_quantize_rht(P(x), s, s, fp4.BF16, fp4.NVFP4, 0xA5C3, P(codes), P(sc16), P(g), None, P(ws),
+                              ws.numel(), sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    def floor(i):
+        if L.fp4_quantize_ex(P(x), s, s, fp4.BF16, fp4.MXFP4, 32, fp4.QUANT_E8M0_FLOOR, P(codes), P(sc32), P(g), None,
+                             None, None, P(ws), ws.numel(), sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    cases = [("quantize_sr", "train X bf16 [16384, 16384] -> NVFP4 with stochastic rounding (amax + encode; "
+              "one 4-byte random word per element)", sr, 2 * n * 2 + n * 4 + n // 2 + sc16.numel()),
+             ("quantize_rht", "train X bf16 [16384, 16384] -> NVFP4 after the 16-point Hadamard transform "
+              "(transforming amax + encode)", rht, 2 * n * 2 + n // 2 + sc16.numel()),
+             ("quantize_mx_floor", "train X bf16 [16384, 16384] -> MXFP4 with the E8M0 scale rounded down (one pass)",
+              floor, n * 2 + n // 2 + sc32.numel())]
+    out = []
+    for key, name, fn, nbytes in cases:
+        ms, _, clk = timed_batches(fn, max(3, args.steps // 4), args.warmup, di, min_s=0.25)
+        _check(fp4)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"case": name, "ms": ms, "GB/s": gbs, "bytes": nbytes,
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                                 "frac": gbs / peaks["hbm"], "peak_source": peaks["hbm_source"],
+                                 "traffic": traffic_for(key)}, "clocks": clk})
+    del x, rbits, codes, sc16, sc32, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def load_peak_table(dev) -> dict:

@@ -849,17 +849,29 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
       bool released = false;
       if (q * 32 < w.rows_valid && early_release && w.n0 + BN <= p.Nk) {  // warp-uniform
         uint32_t pk[CH / 2];  // this thread's columns [c0, c0 + CH) as scaled BF16 pairs
+        // 32-column TMEM loads, one wait per load: the hand-back of the accumulator
+        // waits for few TMEM round trips
+        constexpr int kLdBatch = CH >= 32 ? 32 : CH;
+        static_assert(CH % kLdBatch == 0 && kLdBatch % 16 == 0, "TMEM load batches");
 #pragma unroll
-        for (int cw = 0; cw < CH; cw += 16) {
-          uint32_t rr[16];
-          tmem_ld16(taddr + c0 + cw, rr);
+        for (int cb = 0; cb < CH; cb += kLdBatch) {
+          uint32_t rr[kLdBatch];
+          if constexpr (kLdBatch % 32 == 0) {
+#pragma unroll
+            for (int h = 0; h < kLdBatch; h += 32) tmem_ld32(taddr + c0 + cb + h, rr + h);
+          } else {
+            tmem_ld16(taddr + c0 + cb, *reinterpret_cast<uint32_t(*)[16]>(rr));
+          }
           tmem_ld_wait();
-          float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]) * scale;
-          if (p.bias || p.act) epi_bias_act(p, row, w.n0 + c0 + cw, v);
+          for (int cw = 0; cw < kLdBatch; cw += 16) {
+            float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) pk[(cw + j) / 2] = pack_bf16x2(v[j], v[j + 1]);
+            for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[cw + j]) * scale;
+            if (p.bias || p.act) epi_bias_act(p, row, w.n0 + c0 + cb + cw, v);
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) pk[(cb + cw + j) / 2] = pack_bf16x2(v[j], v[j + 1]);
+          }
         }
         tc_fence_before();
         __syncwarp();

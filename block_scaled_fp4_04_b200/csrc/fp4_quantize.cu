@@ -780,7 +780,10 @@ cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float*
 
 template <typename T, int BLOCK, bool MX, int VAR = kQuantPlain>
 static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
-  const int blocks = blocks_for(a.rb_upper * a.ct_count, 8);
+  // one CTA per tile: the hardware starts a new tile as soon as one finishes, which keeps
+  // every SM's loads in flight to the end (a persistent grid would finish in waves, and
+  // leave SMs idle in the last one when the tile count is a few grid sizes)
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(a.rb_upper * a.ct_count, 1 << 30)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(256);
