@@ -497,17 +497,33 @@ def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
     q_codes = torch.empty(m, n // 2, dtype=torch.uint8, device=dev)
     q_scales = torch.empty(fp4.fp4_scales_bytes(m, n, fp4.NVFP4), dtype=torch.uint8, device=dev)
     q_g = torch.tensor([0.05], dtype=torch.float32, device=dev)
+    d_amax = torch.empty(1, dtype=torch.float32, device=dev)
+    # one quantize pass: the activations' global scale supplied by the kernel that produced
+    # them (fp4_gemm_epilogue's amax_out), here computed once before timing
+    gx_in = torch.empty(1, dtype=torch.float32, device=dev)
+    fp4.fp4_amax(xd, m * k, fp4.BF16, d_amax, ws, wn)
+    fp4.fp4_global_scale(d_amax, gx_in)
+
+    def step_one_pass(i):
+        q = wq[i % copies]
+        if L.fp4_quantize(P(xd), m, k, fp4.BF16, fp4.NVFP4, 16, P(xc), P(xs), P(xg), None, None, P(gx_in), P(ws),
+                          wn, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+        if L.fp4_gemm_ex(fp4.NVFP4, P(xc), P(xs), P(xg), P(q.codes), P(q.scales), P(q.g), m, n, k, P(d), fp4.BF16,
+                         P(ws), wn, fp4.GEMM_WEIGHTS_READY, sp):
+            raise RuntimeError(fp4.fp4_last_error())
 
     def gemm_epi(i):
         q = wq[i % copies]
         if L.fp4_gemm_epilogue(fp4.NVFP4, P(xc), P(xs), P(xg), P(q.codes), P(q.scales), P(q.g), m, n, k, P(bias),
-                               fp4.ACT_RELU, P(d), fp4.BF16, P(q_codes), P(q_scales), P(q_g), P(ws), wn, sp):
+                               fp4.ACT_RELU, P(d), fp4.BF16, P(q_codes), P(q_scales), P(q_g), P(d_amax), P(ws), wn, sp):
             raise RuntimeError(fp4.fp4_last_error())
 
     di = dev.index or 0
     step_ms, batches, clk = timed_batches(step, args.steps, args.warmup, di)
     gemm_ms, _, gclk = timed_batches(gemm, args.steps, args.warmup, di)
     epi_ms, _, eclk = timed_batches(gemm_epi, args.steps, args.warmup, di)
+    one_ms, _, oclk = timed_batches(step_one_pass, args.steps, args.warmup, di)
     _check(fp4)
     flop = 2.0 * m * n * k
     x_host = x.pin_memory()
@@ -526,7 +542,11 @@ def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
                                         "prefill_gemm", {"gemm_clocks": gclk}),
            "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                    "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2},
-           "epilogue_gemm": {"what": "fp4_gemm_epilogue: + bias, ReLU, BF16 out and an NVFP4 copy of the result",
+           "step_one_pass": {"what": "quantize X in one pass with its global scale supplied by the kernel that "
+                                     "produced X (fp4_gemm_epilogue's amax_out), then the GEMM (2 launches)",
+                             "ms": one_ms, "TFLOP/s": flop / (one_ms * 1e-3) / 1e12, "clocks": oclk},
+           "epilogue_gemm": {"what": "fp4_gemm_epilogue: + bias, ReLU, BF16 out, an NVFP4 copy of the result and "
+                                     "its amax",
                              "ms": epi_ms, "TFLOP/s": flop / (epi_ms * 1e-3) / 1e12,
                              "frac": flop / (epi_ms * 1e-3) / 1e12 / peaks["fp4"], "clocks": eclk,
                              "traffic": traffic_for("prefill_gemm_epilogue")},
@@ -542,7 +562,7 @@ def measure_prefill(args, dev, peaks, cpu: bool) -> dict:
         rec["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                "sample": f"{reps} x (quantize {rows} rows of X with the tensor's g, FP64 product "
                                          f"with the 8192 x 8192 dequantized weights)"}
-    del wq, xd, xc, xs, ws, d, x_stage, q_codes, q_scales, bias
+    del wq, xd, xc, xs, ws, d, x_stage, q_codes, q_scales, bias, d_amax, gx_in
     torch.cuda.empty_cache()
     return rec
 

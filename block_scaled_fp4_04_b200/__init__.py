@@ -70,8 +70,8 @@ def lib() -> ctypes.CDLL:
                 "fp4_gemm_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_noalloc": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
                 "fp4_gemm_epilogue_workspace_size": (SZ, [I64, I64, I64, I32, I32]),
-                "fp4_gemm_epilogue": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, I32, P, P, P, P, SZ,
-                                            P]),
+                "fp4_gemm_epilogue": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, I32, P, P, P, P, P,
+                                            SZ, P]),
                 "fp4_gemm_bf16a_workspace_size": (SZ, [I64, I64, I64]),
                 "fp4_gemm_bf16a": (I32, [P, P, P, P, I64, I64, I64, P, I32, P, P, P, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_grouped": (I32, [I32, I32, P, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
@@ -200,15 +200,15 @@ def fp4_gemm_ex(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, workspace=None
                              _p(workspace), workspace_bytes, flags, _s(stream)))
 
 
-def fp4_gemm_epilogue_workspace_size(M: int, N: int, K: int, fmt: int, fp4_out: bool) -> int:
-    return int(lib().fp4_gemm_epilogue_workspace_size(M, N, K, fmt, 1 if fp4_out else 0))
+def fp4_gemm_epilogue_workspace_size(M: int, N: int, K: int, fmt: int, rows_in_place: bool) -> int:
+    return int(lib().fp4_gemm_epilogue_workspace_size(M, N, K, fmt, 1 if rows_in_place else 0))
 
 
 def fp4_gemm_epilogue(fmt, A, sA, gA, B, sB, gB, M, N, K, bias, act, D, out_dtype, Dcodes=None, Dscales=None,
-                      gD=None, workspace=None, workspace_bytes=0, stream=None):
+                      gD=None, amax_out=None, workspace=None, workspace_bytes=0, stream=None):
     _check(lib().fp4_gemm_epilogue(fmt, _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB), M, N, K, _p(bias), act, _p(D),
-                                   out_dtype, _p(Dcodes), _p(Dscales), _p(gD), _p(workspace), workspace_bytes,
-                                   _s(stream)))
+                                   out_dtype, _p(Dcodes), _p(Dscales), _p(gD), _p(amax_out), _p(workspace),
+                                   workspace_bytes, _s(stream)))
 
 
 def fp4_gemm_bf16a_workspace_size(M: int, N: int, K: int) -> int:

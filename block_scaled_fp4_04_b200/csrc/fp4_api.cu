@@ -304,7 +304,8 @@ fp4_status fp4_gemm(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const floa
 fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, const float* gA, const uint8_t* B,
                              const uint8_t* sB, const float* gB, int64_t M, int64_t N, int64_t K, const float* bias,
                              fp4_act act, void* D, fp4_dtype out_dtype, uint8_t* Dcodes, uint8_t* Dscales,
-                             const float* gD, void* workspace, size_t workspace_bytes, void* stream) {
+                             const float* gD, float* amax_out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
   if (act != FP4_ACT_NONE && act != FP4_ACT_RELU) return fail(FP4_ERR_INVALID_ARG, "act");
   if (!D && !Dcodes) return fail(FP4_ERR_INVALID_ARG, "no output: D and Dcodes are both NULL");
   if (Dcodes && (!Dscales || !gD)) return fail(FP4_ERR_INVALID_ARG, "FP4 output needs Dscales and gD");
@@ -331,6 +332,12 @@ fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, c
   g.q_codes = Dcodes;
   g.q_scales = Dscales;
   g.q_g = gD;
+  g.amax_out = amax_out;
+  if (amax_out) {
+    if (reinterpret_cast<uintptr_t>(amax_out) & 3u) return fail(FP4_ERR_INVALID_ARG, "amax_out alignment");
+    const cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "zeroing amax_out");
+  }
   if (Dcodes && (M % 128 != 0 || (N / 16) % 4 != 0)) {
     // the kernel writes the scale bytes of real rows and blocks; the layout's pad bytes
     // (rows up to a multiple of 128, block columns up to a multiple of 4) must read as 0
@@ -341,9 +348,9 @@ fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A, const uint8_t* sA, c
   return gemm_common(g, fmt, out_dtype, stream);
 }
 
-size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int fp4_out) {
+size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int rows_in_place) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  return gemm_workspace_bytes(M, N, K, fmt == FP4_MXFP4, fp4_out != 0);
+  return gemm_workspace_bytes(M, N, K, fmt == FP4_MXFP4, rows_in_place != 0);
 }
 
 size_t fp4_gemm_bf16a_workspace_size(int64_t M, int64_t N, int64_t K) {

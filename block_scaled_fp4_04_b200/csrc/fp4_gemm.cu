@@ -91,6 +91,7 @@ struct GemmArgs {
   uint8_t* q_scales;   // swizzled scale atoms of the [M, N/16] block scales
   const float* q_g;    // global scale of the NVFP4 result (device)
   int64_t q_atoms;     // scale atoms per 128-row block of the result: ceil(N/16, 4) / 4
+  unsigned* amax_out;  // max |result| as float bits (zeroed before the launch), or null
 };
 
 struct Work {
@@ -380,10 +381,15 @@ __device__ __forceinline__ void epi_quantize16(const GemmArgs& p, int row, int c
 
 // Finishes 16 consecutive kernel columns of one kernel row: bias, activation, the
 // BF16 / FP32 store and the NVFP4 copy.
-__device__ __forceinline__ void epi_row16(const GemmArgs& p, int row, int col, float (&v)[16]) {
+__device__ __forceinline__ void epi_row16(const GemmArgs& p, int row, int col, float (&v)[16], uint32_t& tmax) {
   epi_bias_act(p, row, col, v);
   if (p.out) store_row16(p, row, col, v);
   if (p.q_codes && col < p.Nk) epi_quantize16(p, row, col, v);
+  if (p.amax_out) {  // the result's amax, for the global scale of its next quantization
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (p.transposed || col + j < p.Nk) tmax = max(tmax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+  }
 }
 
 // Named barrier among the epilogue threads of one pipeline.
@@ -826,6 +832,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
     };
     wait_prior_grids();               // the global scales come from earlier kernels
     const float ga = p.ga ? *p.ga : 1.0f;
+    uint32_t tmax = 0;                // max |result| over this thread's values (amax_out)
     Sched<BN> sch(p, s_mt, s_off, vb, vg, kMTile, sub_row, s_pt);
     Work w;
     int iter = 0;
@@ -869,6 +876,10 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[cw + j]) * scale;
             if (p.bias || p.act) epi_bias_act(p, row, w.n0 + c0 + cb + cw, v);
+            if (p.amax_out && row_ok) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) tmax = max(tmax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+            }
 #pragma unroll
             for (int j = 0; j < 16; j += 2) pk[(cb + cw + j) / 2] = pack_bf16x2(v[j], v[j + 1]);
           }
@@ -913,7 +924,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]) * scale;
-            epi_row16(p, row, col, v);
+            epi_row16(p, row, col, v, tmax);
           }
         }
         }
@@ -965,12 +976,16 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
                   }
                 }
               }
-              epi_row16(p, row, col, v);
+              epi_row16(p, row, col, v, tmax);
             }
           }
           if (et == 0) p.tile_cnt[w.tile] = 0;
         }
       }
+    }
+    if (p.amax_out) {  // one atomic per warp: non-negative float bits order as integers
+      tmax = __reduce_max_sync(0xFFFFFFFFu, tmax);
+      if (lane == 0 && tmax) atomicMax(p.amax_out, tmax);
     }
   }
 
@@ -1252,7 +1267,7 @@ static cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtenso
 
 int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err) {
   const int grouped = g.num_groups > 0;
-  if (!grouped && !g.mx && !g.q_codes && decode_eligible(g.M, g.N, g.K)) {
+  if (!grouped && !g.mx && !g.q_codes && !g.amax_out && decode_eligible(g.M, g.N, g.K)) {
     // a few activation rows: the decode kernel (the weights are problem B)
     DecodeProblem q{};
     q.W = g.B;
@@ -1274,7 +1289,7 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
     return launch_decode(q, status, st, why, err);
   }
   // the NVFP4 copy of the result is written by rows: keep the operands in place
-  const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx, g.q_codes != nullptr);
+  const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx, g.q_codes != nullptr || g.amax_out != nullptr);
   if (g.ws_bytes < pl.ws_bytes || (pl.ws_bytes && !g.ws)) {
     *why = "workspace too small (see fp4_gemm_workspace_size)";
     return 1;
@@ -1343,6 +1358,7 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
   a.q_scales = g.q_scales;
   a.q_g = g.q_g;
   a.q_atoms = (g.N / 16 + 3) / 4;
+  a.amax_out = reinterpret_cast<unsigned*>(g.amax_out);
   if (pl.mode == kModeStreamK) {
     a.ws = static_cast<float*>(g.ws);
     a.tile_cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(g.ws) + (static_cast<size_t>(g.M * g.N) * 4 + 255) / 256 * 256);

@@ -69,6 +69,7 @@ struct GemmProblem {
   int act;
   uint8_t *q_codes, *q_scales;
   const float* q_g;
+  float* amax_out;  // max |result| (written; zeroed by the entry point), or null
 };
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int mx, bool fp4_out = false);

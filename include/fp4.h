@@ -222,15 +222,20 @@ fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev,
  *           bytes are written as 0, as fp4_quantize writes them.  The result can feed
  *           the next fp4_gemm as its A operand directly.  Needs N % 32 == 0.
  *   bias_dev [N] FP32 or NULL; act FP4_ACT_NONE or FP4_ACT_RELU.
- * workspace: fp4_gemm_epilogue_workspace_size(M, N, K, fmt, Dcodes_dev != NULL) bytes,
- * zero-filled before first use (left zero-filled).  Plain (not grouped) problems only. */
+ *   amax_out_dev: 1 float, or NULL: max |t| over the whole result (zeroed, then written
+ *           by this call), so that the next quantization of t (fp4_global_scale, then
+ *           fp4_quantize with global_in) needs no separate amax pass over it.
+ * workspace: fp4_gemm_epilogue_workspace_size(M, N, K, fmt, rows_in_place) bytes with
+ * rows_in_place = (Dcodes_dev != NULL || amax_out_dev != NULL), zero-filled before first
+ * use (left zero-filled).  Plain (not grouped) problems only. */
 typedef enum { FP4_ACT_NONE = 0, FP4_ACT_RELU = 1 } fp4_act;
-size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int fp4_out);
+size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int rows_in_place);
 fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,
                              const uint8_t* B_dev, const uint8_t* sB_dev, const float* gB_dev,
                              int64_t M, int64_t N, int64_t K, const float* bias_dev, fp4_act act,
                              void* D_dev, fp4_dtype out_dtype, uint8_t* Dcodes_dev, uint8_t* Dscales_dev,
-                             const float* gD_dev, void* workspace_dev, size_t workspace_bytes, void* stream);
+                             const float* gD_dev, float* amax_out_dev, void* workspace_dev,
+                             size_t workspace_bytes, void* stream);
 
 /* BF16-activation GEMM (quantize-on-load): D = gX * gB * (Xq . Bq^T) where Xq is the
  * NVFP4 quantization of the bf16 activations X [M, K] (tensor amax -> gX, 16-blocks,

@@ -219,16 +219,17 @@ def test_gemm_epilogue(m, n, k, act, fp4_out, out_dtype):
     qa, qb = gpu_quantize(xa.cuda(), fp4.NVFP4, 16), gpu_quantize(xb.cuda(), fp4.NVFP4, 16)
     bias = (np.random.default_rng(n).standard_normal(n) * 3.0).astype(np.float32)
     d = torch.empty(m, n, dtype=out_dtype, device="cuda")
-    codes = scales = gD = None
+    codes = scales = gD = amax = None
     if fp4_out:
         codes = torch.empty(m, n // 2, dtype=torch.uint8, device="cuda")
         scales = torch.full((fp4.fp4_scales_bytes(m, n, fp4.NVFP4),), 0xA5, dtype=torch.uint8, device="cuda")
         gD = torch.tensor([0.01], dtype=torch.float32, device="cuda")
+        amax = torch.full((1,), 123.0, dtype=torch.float32, device="cuda")   # zeroed by the call
     wsn = fp4.fp4_gemm_epilogue_workspace_size(m, n, k, fp4.NVFP4, fp4_out)
     ws = torch.zeros(max(wsn, 16), dtype=torch.uint8, device="cuda")
     fp4.fp4_gemm_epilogue(fp4.NVFP4, qa.codes, qa.scales, qa.g, qb.codes, qb.scales, qb.g, m, n, k,
                           torch.from_numpy(bias).cuda(), fp4.ACT_RELU if act == "relu" else fp4.ACT_NONE, d,
-                          fp4.BF16 if out_dtype == torch.bfloat16 else fp4.F32, codes, scales, gD, ws, wsn)
+                          fp4.BF16 if out_dtype == torch.bfloat16 else fp4.F32, codes, scales, gD, amax, ws, wsn)
     torch.cuda.synchronize()
     assert fp4.fp4_get_status() == fp4.OK
     assert not ws.any(), "workspace not left zero-filled"
@@ -239,6 +240,14 @@ def test_gemm_epilogue(m, n, k, act, fp4_out, out_dtype):
     tol = oracle.epilogue_tolerance(t_ref, d_ref, s, bias, out_dtype == torch.bfloat16)
     bad = np.argwhere(~(np.abs(got - t_ref) <= tol))
     assert bad.size == 0, f"{len(bad)} outputs outside tolerance, first {bad[:3].tolist()}"
+    if fp4_out:
+        # the result's amax: exactly the largest stored FP32 magnitude, or the reference's
+        # within the tolerance when the stored copy is BF16
+        if out_dtype == torch.float32:
+            assert amax.item() == float(np.abs(got).max())
+        else:
+            i = np.unravel_index(np.argmax(np.abs(t_ref)), t_ref.shape)
+            assert abs(amax.item() - abs(t_ref[i])) <= tol[i] + 1e-30
     if fp4_out and out_dtype == torch.float32:
         # the NVFP4 copy quantizes the same FP32 values the kernel stored
         oq = oracle.quantize(d.cpu().numpy(), fp4.NVFP4, 16, g_in=np.float32(0.01))
