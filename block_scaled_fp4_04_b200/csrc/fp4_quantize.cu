@@ -281,23 +281,38 @@ struct Quant1DArgs {
   uint32_t signs;          // kQuantRHT: the 16 sign bits of the transform
 };
 
-// One tile = 128 rows x (4 * BLOCK) columns = exactly one 512-byte scale atom.
-// 256 threads; each thread owns one 16-byte chunk per pass; the lanes of one block
-// (BLOCK / elements-per-chunk of them, adjacent) combine their maxima by shuffles.
+// One tile = 128 rows x (4 * BLOCK) columns = exactly one 512-byte scale atom; one CTA of
+// 256 threads per tile.  Each thread owns whole blocks (a row's BLOCK consecutive
+// elements), two per tile: it loads them, takes their maximum, computes the block's scale
+// once, encodes and packs the codes, and stores its scale byte straight into the
+// swizzled atom.  Consecutive threads take consecutive blocks of a row, so a warp reads
+// whole rows of the tile.
+template <typename T>
+struct BlockLoad {
+  static constexpr int kChunks(int block) { return block * static_cast<int>(sizeof(T)) / 16; }
+};
+
+// max |x| over 8 BF16 values packed in a 16-byte chunk, as float bits (NaN propagates:
+// its pattern exceeds every finite one, and so does inf)
+__device__ __forceinline__ uint32_t chunk_absmax_bf16(const uint4& u) {
+  const __nv_bfloat162 a = __hmax2_nan(__habs2(*reinterpret_cast<const __nv_bfloat162*>(&u.x)),
+                                       __habs2(*reinterpret_cast<const __nv_bfloat162*>(&u.y)));
+  const __nv_bfloat162 b = __hmax2_nan(__habs2(*reinterpret_cast<const __nv_bfloat162*>(&u.z)),
+                                       __habs2(*reinterpret_cast<const __nv_bfloat162*>(&u.w)));
+  const __nv_bfloat162 c = __hmax2_nan(a, b);
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(&c);
+  return max(w << 16, w & 0xFFFF0000u);
+}
+
 template <typename T, int BLOCK, bool MX, bool HW, int VAR = kQuantPlain>
 __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int EPC = Elem<T>::kPerChunk;
-  constexpr int TC = 4 * BLOCK;             // columns per tile
-  constexpr int CPR = TC / EPC;             // chunks per tile row
-  constexpr int RPP = 256 / CPR;            // rows per pass
-  constexpr int PASSES = 128 / RPP;
-  constexpr int LPB = BLOCK / EPC;          // lanes per block
-  static_assert(EPC == 4 || EPC == 8, "chunk");
+  constexpr int CH = BLOCK * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per block
+  constexpr int UPT = 2;                                        // blocks per thread per tile
   static_assert(VAR != kQuantMxFloor || MX, "the rounded-down scale is an E8M0 one");
   static_assert(VAR != kQuantSR || (!MX && BLOCK == 16), "stochastic rounding: NVFP4");
-  constexpr int RW = VAR == kQuantSR ? EPC / 4 : 0;  // 16-byte loads of random words per chunk
+  constexpr int RW = VAR == kQuantSR ? BLOCK / 4 : 0;  // 16-byte loads of random words per block
 
-  __shared__ __align__(16) uint8_t s_sf[512];
   __shared__ int s_rb[kMaxGroups + 1];
   __shared__ int s_off[kMaxGroups + 1];
 
@@ -320,9 +335,9 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   if constexpr (!MX) g = *p.g;
 
   const int tid = threadIdx.x;
-  const int chunk = tid % CPR;
   const int64_t half_cols = p.cols / 2;
   const int64_t ntiles = p.rb_upper * p.ct_count;
+  const int64_t nbc = p.cols / BLOCK;  // blocks per row
   unsigned bad = 0;
 
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -346,37 +361,58 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
     }
     const int64_t row_base = s_off[e] + (rb - s_rb[e]) * 128;
     const int64_t row_end = s_off[e + 1];
-    const int64_t col = ct * TC + chunk * EPC;
-    const bool col_ok = col < p.cols;
 
-    uint4 u[PASSES];
-    uint4 rw[PASSES][RW > 0 ? RW : 1];
+    // this thread's blocks: unit q -> row q / 4 of the tile, block column q % 4
+    uint4 u[UPT][CH];
+    uint4 rw[UPT][RW > 0 ? RW : 1];
+    bool ok[UPT];
 #pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int64_t r = row_base + ps * RPP + tid / CPR;
-      if (col_ok && r < row_end)
-        u[ps] = ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + col) * sizeof(T));
-      else
-        u[ps] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < UPT; ++i) {
+      const int q = tid + 256 * i;
+      const int64_t r = row_base + (q >> 2);
+      const int64_t bcol = ct * 4 + (q & 3);
+      ok[i] = r < row_end && bcol < nbc;
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) +
+                                                        (r * p.cols + bcol * BLOCK) * static_cast<int64_t>(sizeof(T)));
+#pragma unroll
+      for (int c = 0; c < CH; ++c) u[i][c] = ok[i] ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
       if constexpr (RW > 0) {
+        const uint4* rsrc = reinterpret_cast<const uint4*>(p.rbits + r * p.cols + bcol * BLOCK);
 #pragma unroll
-        for (int j = 0; j < RW; ++j)
-          rw[ps][j] = (col_ok && r < row_end) ? ld_stream(p.rbits + r * p.cols + col + 4 * j) : make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < RW; ++c) rw[i][c] = ok[i] ? ld_stream(rsrc + c) : make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int rl = ps * RPP + tid / CPR;  // row inside the tile
+    for (int i = 0; i < UPT; ++i) {
+      const int q = tid + 256 * i;
+      const int rl = q >> 2, bc = q & 3;
       const int64_t r = row_base + rl;
-      float v[EPC];
-      Elem<T>::unpack(u[ps], v);
-      if constexpr (VAR == kQuantRHT) rht16_lanes<EPC>(v, p.signs, (chunk % (16 / EPC)) * EPC);
+      const int64_t bcol = ct * 4 + bc;
+      float v[BLOCK];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        float t[EPC];
+        Elem<T>::unpack(u[i][c], t);
+#pragma unroll
+        for (int j = 0; j < EPC; ++j) v[c * EPC + j] = t[j];
+      }
       uint32_t m = 0;
+      if constexpr (VAR == kQuantRHT) {
 #pragma unroll
-      for (int i = 0; i < EPC; ++i) m = max(m, abs_bits(v[i]));
+        for (int h = 0; h < BLOCK; h += 16) {
+          float (&w16)[16] = *reinterpret_cast<float(*)[16]>(v + h);
+          rht16_lanes<16>(w16, p.signs, 0);
+        }
 #pragma unroll
-      for (int d = 1; d < LPB; d <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
-      bad |= m >= 0x7F800000u;
+        for (int j = 0; j < BLOCK; ++j) m = max(m, abs_bits(v[j]));
+      } else if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) m = max(m, chunk_absmax_bf16(u[i][c]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < BLOCK; ++j) m = max(m, abs_bits(v[j]));
+      }
+      bad |= ok[i] && m >= 0x7F800000u;
       const float amax_b = __uint_as_float(m);
       uint32_t sb;
       float mul;
@@ -386,45 +422,38 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       } else {
         mul = nvfp4_block_scale(amax_b, g, sb);
       }
-      float s[EPC];
+      const bool inf_mul = !MX && isinf(mul);  // 1/denom overflowed: zeros stay zeros, not NaN
+      uint32_t packed[BLOCK / 8];
 #pragma unroll
-      for (int i = 0; i < EPC; ++i) s[i] = __fmul_rn(v[i], mul);
-      if constexpr (!MX) {
-        if (isinf(mul)) {  // 1/denom overflowed (denom < 2^-128): zeros stay zeros, not NaN
+      for (int o = 0; o < BLOCK / 8; ++o) {
+        float sv[8];
 #pragma unroll
-          for (int i = 0; i < EPC; ++i)
-            if (v[i] == 0.0f) s[i] = v[i];
+        for (int j = 0; j < 8; ++j) {
+          const float x = v[o * 8 + j];
+          sv[j] = (inf_mul && x == 0.0f) ? x : __fmul_rn(x, mul);
         }
-      }
-      const bool ok = col_ok && r < row_end;
-      if constexpr (VAR == kQuantSR) {
-        uint32_t packed = 0;
+        if constexpr (VAR == kQuantSR) {
+          uint32_t word = 0;
 #pragma unroll
-        for (int i = 0; i < EPC; ++i) {
-          const uint4 w4 = rw[ps][i / 4];
-          const uint32_t bits = (i & 3) == 0 ? w4.x : (i & 3) == 1 ? w4.y : (i & 3) == 2 ? w4.z : w4.w;
-          packed |= e2m1_code_sr(s[i], bits) << (4 * i);
-        }
-        if constexpr (EPC == 8) {
-          if (ok) *reinterpret_cast<uint32_t*>(p.codes + r * half_cols + col / 2) = packed;
+          for (int j = 0; j < 8; ++j) {
+            const uint4 w4 = rw[i][(o * 8 + j) / 4];
+            const int k = (o * 8 + j) & 3;
+            const uint32_t bits = k == 0 ? w4.x : k == 1 ? w4.y : k == 2 ? w4.z : w4.w;
+            word |= e2m1_code_sr(sv[j], bits) << (4 * j);
+          }
+          packed[o] = word;
         } else {
-          if (ok) *reinterpret_cast<uint16_t*>(p.codes + r * half_cols + col / 2) = static_cast<uint16_t>(packed);
+          packed[o] = pack8<HW>(sv);
         }
-      } else if constexpr (EPC == 8) {
-        const uint32_t packed = pack8<HW>(s);
-        if (ok) *reinterpret_cast<uint32_t*>(p.codes + r * half_cols + col / 2) = packed;
-      } else {
-        const uint32_t packed = pack4<HW>(s);
-        if (ok) *reinterpret_cast<uint16_t*>(p.codes + r * half_cols + col / 2) = static_cast<uint16_t>(packed);
       }
-      if (chunk % LPB == 0) {
-        const int bc = chunk / LPB;  // block column inside the atom (0..3)
-        s_sf[(rl & 31) * 16 + (rl >> 5) * 4 + bc] = ok ? static_cast<uint8_t>(sb) : 0;
+      if (ok[i]) {
+        uint8_t* dst = p.codes + r * half_cols + bcol * (BLOCK / 2);
+        if constexpr (BLOCK == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
+      // the scale byte at its place in the atom (rows and blocks past the tensor: 0)
+      atom[(rl & 31) * 16 + (rl >> 5) * 4 + bc] = ok[i] ? static_cast<uint8_t>(sb) : 0;
     }
-    __syncthreads();
-    if (tid < 32) reinterpret_cast<uint4*>(atom)[tid] = reinterpret_cast<const uint4*>(s_sf)[tid];
-    __syncthreads();
   }
   if (bad) atomicOr(p.status, kStatusNonFinite);
 }
