@@ -44,14 +44,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// A thread whose phase is not complete may be suspended for up to kWaitSuspendNs, and is
+// woken early when the phase completes.  A suspended waiter issues nothing, which leaves the
+// SM sub-partition's issue slots to the threads on the critical path (the TMA producer, the
+// MMA issuer).  Measured on the decode kernel and the persistent GEMM against the same
+// kernels without the hint: +5% and +2-4% throughput.
+constexpr uint32_t kWaitSuspendNs = 1000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitSuspendNs)
       : "memory");
   return ok != 0;
 }
