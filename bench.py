@@ -688,7 +688,7 @@ def measure_moe(args, dev, peaks, cpu: bool) -> dict:
                       "step": "grouped MXFP4 quantize of the activations + grouped GEMM (2 launches)",
                       "l2": "expert weights (265 MiB) exceed the L2"},
            "roofline": {"bound": "tensor" if flop / peaks["fp4"] * 1e-9 > gemm_bytes / peaks["hbm"] else "hbm",
-                        "kernel": "fp4_gemm_kernel<256, mxfp4, 1 acc, CTA pair> (grouped)",
+                        "kernel": "fp4_gemm_kernel<256, mxfp4, 1 acc> (grouped, 128-row tiles)",
                         "achieved": achieved, "peak": peaks["fp4"], "unit": "TFLOP/s",
                         "frac": t_roof_ms / gemm_ms,
                         "frac_definition": "roofline time (slower of tensor and HBM) / measured kernel time",

@@ -1126,18 +1126,24 @@ struct Plan {
   size_t ws_bytes;
 };
 
-static Plan make_plan(int64_t M, int64_t N, int64_t K, int grouped, int mx, bool row_major_out = false) {
+// `groups` is the number of experts of a grouped problem, 0 for a plain GEMM.
+static Plan make_plan(int64_t M, int64_t N, int64_t K, int groups, int mx, bool row_major_out = false) {
   Plan pl{};
   pl.num_kb = static_cast<int>((K + 255) / 256);
   (void)mx;
-  if (grouped) {
+  if (groups) {
     // 256-wide tiles: per MMA the scale-factor copies into TMEM cost less than with
     // 128-wide ones (an expert's last N-tile may be half empty; its extra columns, read
     // from the next expert's rows, are never stored)
     pl.swap = false;
     pl.BN = N >= 256 ? 256 : 128;
     pl.ACC = pl.BN == 256 ? 1 : 2;
-    pl.pair = pl.BN == 256;  // 256 x 256 tiles (per expert) on CTA pairs
+    // 256 x 256 tiles on CTA pairs load a third fewer bytes per MMA, but an expert's last
+    // row tile is on average half empty: 128 rows of padding per expert instead of 64.
+    // With experts of a few hundred rows (top-k routing of a few thousand tokens) the
+    // padding costs more than the pairs save (measured on 32 experts of ~512 rows:
+    // 128-row tiles 5% faster per clock); pairs from 1280 rows per expert on average.
+    pl.pair = pl.BN == 256 && M >= 1280 * static_cast<int64_t>(groups);
     pl.mode = kModeGrouped;
     pl.Mk = M;
     pl.Nk = N;
@@ -1289,7 +1295,7 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
     return launch_decode(q, status, st, why, err);
   }
   // the NVFP4 copy of the result is written by rows: keep the operands in place
-  const Plan pl = make_plan(g.M, g.N, g.K, grouped, g.mx, g.q_codes != nullptr || g.amax_out != nullptr);
+  const Plan pl = make_plan(g.M, g.N, g.K, g.num_groups, g.mx, g.q_codes != nullptr || g.amax_out != nullptr);
   if (g.ws_bytes < pl.ws_bytes || (pl.ws_bytes && !g.ws)) {
     *why = "workspace too small (see fp4_gemm_workspace_size)";
     return 1;

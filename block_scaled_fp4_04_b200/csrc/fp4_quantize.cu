@@ -603,93 +603,90 @@ struct Quant2DArgs {
   unsigned* status;
 };
 
-// One CTA per 128 x 128 region of W (rows and cols beyond the tensor are zero).  The
-// region is staged in shared memory (FP32, padded rows); 64 16x16 patches give 64 scale
-// bytes; then W's codes are written row-wise and W^T's codes column-wise, and both
-// scale layouts receive two full 512-byte atoms per region.
+// Four consecutive elements of one row, as FP32 (16-byte load for FP32, 8-byte for BF16).
+template <typename T>
+__device__ __forceinline__ void load4(const T* src, float (&v)[4]);
+template <>
+__device__ __forceinline__ void load4<float>(const float* src, float (&v)[4]) {
+  const uint4 u = ld_stream(src);
+  v[0] = __uint_as_float(u.x);
+  v[1] = __uint_as_float(u.y);
+  v[2] = __uint_as_float(u.z);
+  v[3] = __uint_as_float(u.w);
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* src, float (&v)[4]) {
+  uint32_t a, b;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(a), "=r"(b) : "l"(src));
+  v[0] = __uint_as_float(a << 16);
+  v[1] = __uint_as_float(a & 0xFFFF0000u);
+  v[2] = __uint_as_float(b << 16);
+  v[3] = __uint_as_float(b & 0xFFFF0000u);
+}
+
+// One CTA per 128 x 128 region of W; warp w holds the region's 16-row band w in registers,
+// lane l its four columns 4l .. 4l+3, so that the four lanes of a 16 x 16 patch find the
+// patch amax with two shuffles.  Each element's ratio to its patch scale is formed once and
+// encoded twice: in row pairs along W's rows (W's codes) and in pairs down the columns
+// (W^T's codes, eight bytes per column of the band).  The patches' scale bytes meet in
+// shared memory, and both scale layouts receive two full 512-byte atoms per region.  Rows
+// (a multiple of 32) and columns (a multiple of 32) beyond the tensor are zero: a band and a
+// lane's four columns are either wholly inside or wholly outside.
 template <typename T, bool HW>
-__global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
-  extern __shared__ __align__(16) float s_x[];  // [128][129]
+__global__ void __launch_bounds__(256, 3) quantize_2d_kernel(const Quant2DArgs p) {
   __shared__ uint8_t s_sb[8][8];
-  __shared__ float s_mul[8][8];
   __shared__ __align__(16) uint8_t s_atom[2][512];
-  constexpr int LD = 129;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 128;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const int64_t rb = r0 + warp * 16;  // this warp's first row
+  const int64_t cl = c0 + lane * 4;   // this lane's first column
+  const bool in = rb < p.rows && cl < p.cols;
   const float g = *p.g;
-  constexpr int EPC = Elem<T>::kPerChunk;
-  constexpr int CPR = 128 / EPC;
-  unsigned bad = 0;
 
-  // stage the region, eight 16-byte loads in flight per thread
-  constexpr int NLD = 8;
-  static_assert((128 * CPR) % (256 * NLD) == 0, "staging loop");
-  for (int base = tid; base < 128 * CPR; base += 256 * NLD) {
-    uint4 u[NLD];
+  float v[16][4];
+  if (in) {
+    const T* src = static_cast<const T*>(p.x) + rb * p.cols + cl;
 #pragma unroll
-    for (int j = 0; j < NLD; ++j) {
-      const int idx = base + j * 256;
-      const int rl = idx / CPR, ch = idx % CPR;
-      const int64_t r = r0 + rl, c = c0 + ch * EPC;
-      u[j] = (r < p.rows && c < p.cols) ? ld_stream(static_cast<const uint8_t*>(p.x) + (r * p.cols + c) * sizeof(T))
-                                        : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 16; ++i) load4<T>(src + i * p.cols, v[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.0f;
+  }
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = max(m, abs_bits(v[i][j]));
+  m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+  m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+  const unsigned bad = m >= 0x7F800000u;
+  uint32_t sb;
+  const float mul = nvfp4_block_scale(__uint_as_float(m), g, sb);
+  if ((lane & 3) == 0) s_sb[warp][lane >> 2] = static_cast<uint8_t>(sb);
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[i][j] = ratio(v[i][j], mul);
+  if (in) {
+    // W: two rows per pack8 (four codes of each), sixteen bits per row and lane
+    uint8_t* wrow = p.codes + rb * (p.cols / 2) + cl / 2;
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float a[8] = {v[i][0], v[i][1], v[i][2], v[i][3], v[i + 1][0], v[i + 1][1], v[i + 1][2], v[i + 1][3]};
+      const uint32_t w = pack8<HW>(a);
+      *reinterpret_cast<uint16_t*>(wrow + i * (p.cols / 2)) = static_cast<uint16_t>(w);
+      *reinterpret_cast<uint16_t*>(wrow + (i + 1) * (p.cols / 2)) = static_cast<uint16_t>(w >> 16);
     }
+    // W^T: column j of the band is sixteen codes, eight bytes of W^T's row cl + j
 #pragma unroll
-    for (int j = 0; j < NLD; ++j) {
-      const int idx = base + j * 256;
-      const int rl = idx / CPR, ch = idx % CPR;
-      float v[EPC];
-      Elem<T>::unpack(u[j], v);
-#pragma unroll
-      for (int i = 0; i < EPC; ++i) s_x[rl * LD + ch * EPC + i] = v[i];
+    for (int j = 0; j < 4; ++j) {
+      const float a[8] = {v[0][j], v[1][j], v[2][j], v[3][j], v[4][j], v[5][j], v[6][j], v[7][j]};
+      const float b[8] = {v[8][j], v[9][j], v[10][j], v[11][j], v[12][j], v[13][j], v[14][j], v[15][j]};
+      *reinterpret_cast<uint2*>(p.codesT + (cl + j) * (p.rows / 2) + rb / 2) = make_uint2(pack8<HW>(a), pack8<HW>(b));
     }
   }
   __syncthreads();
-  // patch amax: 4 threads per patch, 4 rows each
-  {
-    const int patch = tid >> 2, sub = tid & 3;
-    const int pr = patch >> 3, pc = patch & 7;
-    uint32_t m = 0;
-    for (int i = 0; i < 4; ++i)
-      for (int j = 0; j < 16; ++j) m = max(m, abs_bits(s_x[(pr * 16 + sub * 4 + i) * LD + pc * 16 + j]));
-    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    bad |= m >= 0x7F800000u;
-    if (sub == 0) {
-      uint32_t sb;
-      s_mul[pr][pc] = nvfp4_block_scale(__uint_as_float(m), g, sb);
-      s_sb[pr][pc] = static_cast<uint8_t>(sb);
-    }
-  }
-  __syncthreads();
-  // W codes: thread -> (row, 16-column block); W^T codes: thread -> (col, 16-row block)
-  for (int idx = tid; idx < 128 * 8; idx += 256) {
-    const int rl = idx >> 3, bc = idx & 7;
-    const float mul = s_mul[rl >> 4][bc];
-    float a[8], b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      a[i] = ratio(s_x[rl * LD + bc * 16 + i], mul);
-      b[i] = ratio(s_x[rl * LD + bc * 16 + 8 + i], mul);
-    }
-    const int64_t r = r0 + rl, c = c0 + bc * 16;
-    const uint2 w = make_uint2(pack8<HW>(a), pack8<HW>(b));
-    if (r < p.rows && c < p.cols) *reinterpret_cast<uint2*>(p.codes + r * (p.cols / 2) + c / 2) = w;
-  }
-  for (int idx = tid; idx < 128 * 8; idx += 256) {
-    const int cl = idx & 127, br = idx >> 7;  // consecutive threads -> consecutive columns
-    const float mul = s_mul[br][cl >> 4];
-    float a[8], b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      a[i] = ratio(s_x[(br * 16 + i) * LD + cl], mul);
-      b[i] = ratio(s_x[(br * 16 + 8 + i) * LD + cl], mul);
-    }
-    const int64_t c = c0 + cl, r = r0 + br * 16;
-    const uint2 w = make_uint2(pack8<HW>(a), pack8<HW>(b));
-    if (c < p.cols && r < p.rows) *reinterpret_cast<uint2*>(p.codesT + c * (p.rows / 2) + r / 2) = w;
-  }
   // scale atoms.  W: rows r0..r0+127, scale columns c0/16 .. +7 -> atoms (r0/128, c0/64 + {0,1}).
   // W^T: rows c0..c0+127, scale columns r0/16 .. +7 -> atoms (c0/128, r0/64 + {0,1}).
   for (int pass = 0; pass < 2; ++pass) {
@@ -697,10 +694,10 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
       const int a = idx >> 9, rem = idx & 511, rl = rem >> 2, cc = rem & 3;
       const int off = (rl & 31) * 16 + (rl >> 5) * 4 + cc;
       const int b = a * 4 + cc;  // scale column inside the region (0..7)
-      uint8_t v;
-      if (pass == 0) v = ((r0 + rl) < p.rows && (c0 + b * 16) < p.cols) ? s_sb[rl >> 4][b] : 0;
-      else v = ((c0 + rl) < p.cols && (r0 + b * 16) < p.rows) ? s_sb[b][rl >> 4] : 0;
-      s_atom[a][off] = v;
+      uint8_t byte;
+      if (pass == 0) byte = ((r0 + rl) < p.rows && (c0 + b * 16) < p.cols) ? s_sb[rl >> 4][b] : 0;
+      else byte = ((c0 + rl) < p.cols && (r0 + b * 16) < p.rows) ? s_sb[b][rl >> 4] : 0;
+      s_atom[a][off] = byte;
     }
     __syncthreads();
     const int64_t natoms = pass == 0 ? ((p.cols / 16) + 3) / 4 : ((p.rows / 16) + 3) / 4;
@@ -708,7 +705,7 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(const Quant2DArgs p) {
     const int64_t first = pass == 0 ? c0 / 64 : r0 / 64;
     uint8_t* dst = pass == 0 ? p.scales : p.scalesT;
     if (tid < 64) {
-      const int a = tid >> 5, lane = tid & 31;
+      const int a = tid >> 5;
       if (first + a < natoms)
         reinterpret_cast<uint4*>(dst + (rowblk * natoms + first + a) * 512)[lane] =
             reinterpret_cast<const uint4*>(s_atom[a])[lane];
@@ -911,19 +908,10 @@ cudaError_t launch_quantize_2d(const void* x, int64_t rows, int64_t cols, int bf
                                unsigned* status, cudaStream_t st) {
   Quant2DArgs a{x, rows, cols, codes, scales, codesT, scalesT, g, status};
   dim3 grid(static_cast<unsigned>((cols + 127) / 128), static_cast<unsigned>((rows + 127) / 128));
-  const size_t smem = 128 * 129 * sizeof(float);
-  cudaError_t e;
-  if (bf16) {
-    e = cudaFuncSetAttribute(quantize_2d_kernel<__nv_bfloat16, kE2M1Hardware>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    quantize_2d_kernel<__nv_bfloat16, kE2M1Hardware><<<grid, 256, smem, st>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(quantize_2d_kernel<float, kE2M1Hardware>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    quantize_2d_kernel<float, kE2M1Hardware><<<grid, 256, smem, st>>>(a);
-  }
+  if (bf16)
+    quantize_2d_kernel<__nv_bfloat16, kE2M1Hardware><<<grid, 256, 0, st>>>(a);
+  else
+    quantize_2d_kernel<float, kE2M1Hardware><<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -177,12 +177,18 @@ def test_split_k_counters_reset_between_shapes():
         check_gemm(d, dequant_oracle(oa, fp4.NVFP4), dequant_oracle(ob, fp4.NVFP4), label=f"{m}x{n}x{k}")
 
 
-@pytest.mark.parametrize("N", [256, 384, 128])
-def test_grouped_gemm_moe_small(N):
+SMALL_EXPERTS = (0, 130, 130, 300, 301, 560)
+LARGE_EXPERTS = (0, 1300, 1300, 4000)   # >= 1280 rows per expert on average: CTA-pair tiles
+
+
+@pytest.mark.parametrize("offs,N", [(SMALL_EXPERTS, 256), (SMALL_EXPERTS, 384), (SMALL_EXPERTS, 128),
+                                    (LARGE_EXPERTS, 256), (LARGE_EXPERTS, 384)])
+def test_grouped_gemm_moe_small(offs, N):
     """Grouped MXFP4 GEMM with an empty expert and ragged expert sizes; N = 384 leaves each
     expert's last 256-wide tile half empty (it reads into the next expert's weights, and
-    past the last expert's, without storing those columns)."""
-    offsets = np.array([0, 130, 130, 300, 301, 560], np.int32)
+    past the last expert's, without storing those columns).  Small experts run 128-row
+    tiles on single CTAs, large ones 256-row tiles on CTA pairs (partly empty last tiles)."""
+    offsets = np.array(offs, np.int32)
     E, K = len(offsets) - 1, 2880
     rows = int(offsets[-1])
     xa = random_input(rows, K, 41, torch.bfloat16)

@@ -36,11 +36,22 @@ def test_quantize_1d_bit_exact(rows, cols, dtype, fmt, block):
 
 
 @pytest.mark.parametrize("rows,cols,dtype", [(32, 32, torch.float32), (64, 96, torch.bfloat16),
-                                             (160, 128, torch.float32), (288, 320, torch.bfloat16)])
+                                             (160, 128, torch.float32), (288, 320, torch.bfloat16),
+                                             # partial last regions in both directions
+                                             (416, 544, torch.float32), (1056, 2080, torch.bfloat16)])
 def test_quantize_2d_bit_exact(rows, cols, dtype):
     x = random_input(rows, cols, rows + 3 * cols, dtype, std=0.02)
     gq = gpu_quantize(x.cuda(), fp4.NVFP4, 256)
     assert_quant_equal(gq, oracle_quantize(x, fp4.NVFP4, 256), f"2d {rows}x{cols}")
+
+
+def test_quantize_2d_nonfinite_with_caller_global_scale():
+    # with a caller g there is no amax pass: the 2-D kernel's own patch check reports it
+    x = torch.ones(96, 160)
+    x[70, 133] = float("inf")
+    fp4.fp4_get_status()
+    gpu_quantize(x.cuda(), fp4.NVFP4, 256, g_in=0.25)
+    assert fp4.fp4_get_status() == fp4.ERR_NONFINITE
 
 
 def test_quantize_caller_global_scale():
