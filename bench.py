@@ -242,6 +242,7 @@ def run_decode(args, dist: Dist, dev):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     batch_ms, total_ms = [], 0.0
+    min_ms = 500.0 if MIN_S_OVERRIDE is None else MIN_S_OVERRIDE * 1e3
     c0 = clocks.mark()
     while True:
         dist.barrier()
@@ -255,7 +256,7 @@ def run_decode(args, dist: Dist, dev):
         b = dist.max(t_start.elapsed_time(t_end), dev)
         batch_ms.append(b)
         total_ms += b
-        if total_ms >= 500.0 and len(batch_ms) >= 3:
+        if total_ms >= min_ms and len(batch_ms) >= 3:
             break
     c1 = clocks.mark()
     clk = clocks.stop(c0, c1)
@@ -354,6 +355,7 @@ def run_decode(args, dist: Dist, dev):
 # ---------------------------------------------------------------- the other configurations
 FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 MIN_TIMED_S = 0.4   # each sub-workload is timed over at least this long (clock samples cover it)
+MIN_S_OVERRIDE = None  # --min-seconds: one minimum for every timed loop (short runs under a profiler)
 
 
 def _check(fp4):
@@ -376,6 +378,8 @@ def timed_batches(fn, steps: int, warmup: int, dev_index: int, min_s: float = MI
     clocks = ClockSampler(dev_index)
     time.sleep(0.15)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if MIN_S_OVERRIDE is not None:
+        min_s = MIN_S_OVERRIDE
     batches, total, i = [], 0.0, 0
     c0 = clocks.mark()
     while total < min_s * 1e3 or len(batches) < 3:
@@ -744,6 +748,8 @@ def measure_quantize(args, dev, peaks, cpu: bool) -> dict:
     cases[1] = cases[1][:2] + (lambda: train_tensor(0),) + cases[1][3:]
     cases[3] = cases[3][:2] + (lambda: train_tensor(1),) + cases[3][3:]
     for key, name, make, fmt, blk in cases:
+        if args.case and key != args.case:
+            continue
         xh = make()
         x = xh.to(dev)
         rows, cols = x.shape
@@ -781,7 +787,8 @@ def measure_quantize(args, dev, peaks, cpu: bool) -> dict:
         out.append(rec)
         del x, ws, xh
         torch.cuda.empty_cache()
-    out.extend(measure_quantize_variants(args, dev, peaks, train_tensor))
+    if not args.case or args.case in ("quantize_sr", "quantize_rht", "quantize_mx_floor"):
+        out.extend(measure_quantize_variants(args, dev, peaks, train_tensor))
     return {"cases": out}
 
 
@@ -829,6 +836,8 @@ def measure_quantize_variants(args, dev, peaks, train_tensor) -> list:
               floor, n * 2 + n // 2 + sc32.numel())]
     out = []
     for key, name, fn, nbytes in cases:
+        if args.case and key != args.case:
+            continue
         ms, _, clk = timed_batches(fn, max(3, args.steps // 4), args.warmup, di, min_s=0.25)
         _check(fp4)
         gbs = nbytes / (ms * 1e-3) / 1e9
@@ -939,7 +948,15 @@ def main():
                          "value prints that configuration's record alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the other configurations' sub-records")
+    ap.add_argument("--min-seconds", type=float, default=None,
+                    help="minimum timed duration of every timed loop (default 0.5 s for the step, 0.2-0.4 s for "
+                         "the sub-records); small values keep runs under a profiler short")
+    ap.add_argument("--case", default=None,
+                    help="with --workload quantize: only this case (moe_quantize, quantize_train_x, "
+                         "quantize_decode_w, quantize_2d_w, quantize_sr, quantize_rht, quantize_mx_floor)")
     args = ap.parse_args()
+    global MIN_S_OVERRIDE
+    MIN_S_OVERRIDE = args.min_seconds
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")
     dist = Dist()

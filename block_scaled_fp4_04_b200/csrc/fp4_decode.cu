@@ -362,10 +362,11 @@ __global__ void __launch_bounds__(DecodeCfg<BN>::kThreads, 1)
         return true;
       };
       // later batches that are already quantized: copied after a stage's MMAs are issued,
-      // so that they never delay an MMA that does not need them
+      // so that they never delay an MMA that does not need them (a non-blocking look: a
+      // batch not ready yet must not suspend the MMA thread)
       auto copy_ready = [&]() {
         if (sub != 0) return;
-        while (copied < nbatch && !*s_xfail && mbar_try_wait(&b_ready[copied], 0)) copy_batch(copied++);
+        while (copied < nbatch && !*s_xfail && mbar_test_wait(&b_ready[copied], 0)) copy_batch(copied++);
       };
       auto fail = [&]() {
         if (!*s_xfail) d_latch_timeout(s_abort, p.status);
