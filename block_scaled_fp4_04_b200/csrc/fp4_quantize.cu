@@ -427,10 +427,15 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
 #pragma unroll
       for (int o = 0; o < BLOCK / 8; ++o) {
         float sv[8];
+        if (!inf_mul) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float x = v[o * 8 + j];
-          sv[j] = (inf_mul && x == 0.0f) ? x : __fmul_rn(x, mul);
+          for (int j = 0; j < 8; ++j) sv[j] = __fmul_rn(v[o * 8 + j], mul);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = v[o * 8 + j];
+            sv[j] = x == 0.0f ? x : __fmul_rn(x, mul);
+          }
         }
         if constexpr (VAR == kQuantSR) {
           uint32_t word = 0;
