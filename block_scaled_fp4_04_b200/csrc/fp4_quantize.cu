@@ -108,16 +108,22 @@ __device__ __forceinline__ void rht16_lanes(float (&v)[EPC], uint32_t signs, int
 // two, so the fraction is exact in FP32.  Grid values stay, |s| >= 6 saturates; the sign
 // bit copies s's sign.
 __device__ __forceinline__ uint32_t e2m1_code_sr(float s, uint32_t bits) {
-  const float a = fabsf(s);
-  const uint32_t sign = (__float_as_uint(s) >> 28) & 8u;
-  if (a >= 6.0f) return 7u | sign;
-  const uint32_t lo = (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) + (a >= 4.0f);
-  const float lov = e2m1_value(lo);
-  if (a == lov) return lo | sign;
-  const float inv_gap = lo < 4 ? 2.0f : lo < 6 ? 1.0f : 0.5f;
-  const float frac = __fmul_rn(__fsub_rn(a, lov), inv_gap);
-  const float u = __fmul_rn(__uint2float_rn(bits >> 8), 5.9604644775390625e-08f);  // 2^-24
-  return (u < frac ? lo + 1u : lo) | sign;
+  const uint32_t sb = __float_as_uint(s), ab = sb & 0x7FFFFFFFu;
+  const uint32_t sign = (sb >> 28) & 8u;
+  if (ab > 0x7F800000u) return sign;        // NaN: code 0 (the status word reports it)
+  if (ab >= 0x40C00000u) return 7u | sign;  // |s| >= 6 saturates
+  const uint32_t n = bits >> 8;             // u = n * 2^-24
+  const bool ge1 = ab >= 0x3F800000u;
+  // [1, 6): the lower neighbour's code is 2 + 2 (exponent - 127) + the top mantissa bit, and
+  // the fraction toward the upper one is the 22 mantissa bits below that bit, times 2^-22;
+  // [0.5, 1): the lower neighbour is 0.5 and the fraction the 23 mantissa bits, times 2^-23
+  uint32_t lo = ge1 ? (ab >> 22) - 252u : 1u;
+  bool up = n < (ge1 ? (ab & 0x3FFFFFu) << 2 : (ab & 0x7FFFFFu) << 1);
+  if (ab < 0x3F000000u) {  // [0, 0.5): lower neighbour 0, fraction 2 |s|
+    lo = 0u;
+    up = __fmul_rn(__uint2float_rn(n), 5.9604644775390625e-08f) < __fmul_rn(__uint_as_float(ab), 2.0f);
+  }
+  return (lo + (up ? 1u : 0u)) | sign;
 }
 
 // E8M0 scale rounded down: 2^(floor(log2 amax_b) - 2), i.e. the exponent field less 2,
