@@ -65,6 +65,39 @@ def test_quantize_sr_extreme_words_and_global_in():
         assert_quant_equal(fp4.Quantized(codes, scales, g, rows, cols, fp4.NVFP4), oq, f"word {word:#x}")
 
 
+def test_quantize_sr_words_at_the_decision_boundary():
+    """Every element's random word is placed at its rounding decision: bits >> 8 either the
+    largest value that still rounds up (u just below the fraction) or the one above it.  The
+    fractions are worked out here from round-to-nearest block scales (stochastic rounding
+    keeps them); whether each word lands exactly on the boundary only sharpens the test: the
+    expected codes are the oracle's for those words."""
+    rows, cols = 64, 1024
+    x = random_input(rows, cols, 21, torch.float32)
+    xh = host_input(x)
+    oq = oracle.quantize(xh, fp4.NVFP4, 16)
+    g = np.float32(oq["g"])
+    denom = (np.vectorize(oracle.e4m3_decode)(oq["scales"]).astype(np.float32) * g).astype(np.float32)
+    inv = np.zeros_like(denom)
+    np.divide(np.float32(1.0), denom, out=inv, where=denom != 0)
+    a = np.abs((xh.astype(np.float32) * np.repeat(inv, 16, axis=1)).astype(np.float32))
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    lo = np.clip(np.searchsorted(grid, a, side="right") - 1, 0, 6)
+    frac = (a - grid[lo]).astype(np.float64) / (grid[lo + 1] - grid[lo]).astype(np.float64)
+    rng = np.random.default_rng(22)
+    n = np.ceil(frac * 2 ** 24).astype(np.int64) - 1 + rng.integers(0, 2, a.shape)
+    bits = ((np.clip(n, 0, 2 ** 24 - 1) << 8) | rng.integers(0, 256, a.shape)).astype(np.uint32)
+    codes, scales, gd = _outs(rows, cols, fp4.NVFP4)
+    ws = _ws()
+    fp4.fp4_quantize_sr(x.cuda(), rows, cols, fp4.F32, torch.from_numpy(bits.view(np.int32)).cuda(), codes, scales,
+                        gd, None, ws, ws.numel())
+    assert fp4.fp4_get_status() == fp4.OK
+    osr = oracle.quantize_sr(xh, bits)
+    osr["scales_sw"] = oracle.swizzle_scales(osr["scales"])
+    assert_quant_equal(fp4.Quantized(codes, scales, gd, rows, cols, fp4.NVFP4), osr, "words at the boundary")
+    # the placement did reach both sides of the decision: some codes round up, some do not
+    assert 0 < np.count_nonzero(osr["codes"] != oq["codes"]) < osr["codes"].size
+
+
 def test_quantize_sr_is_unbiased_on_the_device():
     """Averaged over many draws, the dequantized value approaches x (the page's reason for
     stochastic rounding).  In units of the block scale, the per-element error of the mean
