@@ -181,13 +181,15 @@ SMALL_EXPERTS = (0, 130, 130, 300, 301, 560)
 LARGE_EXPERTS = (0, 1300, 1300, 4000)   # >= 1280 rows per expert on average: CTA-pair tiles
 
 
-@pytest.mark.parametrize("offs,N", [(SMALL_EXPERTS, 256), (SMALL_EXPERTS, 384), (SMALL_EXPERTS, 128),
-                                    (LARGE_EXPERTS, 256), (LARGE_EXPERTS, 384)])
-def test_grouped_gemm_moe_small(offs, N):
+@pytest.mark.parametrize("offs,N,out", [(SMALL_EXPERTS, 256, "bf16"), (SMALL_EXPERTS, 384, "bf16"),
+                                        (SMALL_EXPERTS, 128, "bf16"), (SMALL_EXPERTS, 384, "f32"),
+                                        (LARGE_EXPERTS, 256, "bf16"), (LARGE_EXPERTS, 384, "bf16")])
+def test_grouped_gemm_moe_small(offs, N, out):
     """Grouped MXFP4 GEMM with an empty expert and ragged expert sizes; N = 384 leaves each
     expert's last 256-wide tile half empty (it reads into the next expert's weights, and
     past the last expert's, without storing those columns).  Small experts run 128-row
-    tiles on single CTAs, large ones 256-row tiles on CTA pairs (partly empty last tiles)."""
+    tiles on single CTAs, large ones 256-row tiles on CTA pairs (partly empty last tiles).
+    FP32 output takes the epilogue's general path instead of the BF16 row-major one."""
     offsets = np.array(offs, np.int32)
     E, K = len(offsets) - 1, 2880
     rows = int(offsets[-1])
@@ -201,8 +203,9 @@ def test_grouped_gemm_moe_small(offs, N):
     wq = [gpu_quantize(w[e].cuda(), fp4.MXFP4, 32) for e in range(E)]
     B = torch.stack([q.codes for q in wq])
     sB = torch.cat([q.scales for q in wq])
-    D = torch.empty(rows, N, dtype=torch.bfloat16, device="cuda")
-    fp4.fp4_gemm_grouped(fp4.MXFP4, E, off_d, codes, scales, None, B, sB, None, rows, N, K, D, fp4.BF16)
+    D = torch.empty(rows, N, dtype=torch.bfloat16 if out == "bf16" else torch.float32, device="cuda")
+    fp4.fp4_gemm_grouped(fp4.MXFP4, E, off_d, codes, scales, None, B, sB, None, rows, N, K, D,
+                         fp4.BF16 if out == "bf16" else fp4.F32)
     torch.cuda.synchronize()
     assert fp4.fp4_get_status() == fp4.OK
     oa = oracle_quantize(xa, fp4.MXFP4, 32)
