@@ -45,6 +45,7 @@ _lock = threading.Lock()
 
 NVFP4 = 0
 MXFP4 = 1
+MXFP8 = 2  # E4M3 elements, E8M0 scale per 32 (the FP8 operand of the mixed GEMM)
 F32 = 0
 BF16 = 1
 ERR_NONFINITE = 5
@@ -92,6 +93,8 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_scales_bytes_grouped": (I64, [P, I32, I64]),
         "orc_swizzle_scales_grouped": (None, [P, P, I32, I64, P]),
         "orc_dequantize": (None, [P, P, ctypes.c_float, I64, I64, I32, P]),
+        "orc_quantize_mxfp8_1d": (I32, [P, I64, I64, I32, P, P]),
+        "orc_dequantize_mxfp8": (None, [P, P, I64, I64, P]),
         "orc_fake_quant_fp32_scale": (None, [P, I64, I64, P]),
         "orc_e2m1_count_mismatch": (I64, [ctypes.c_uint64, I64, P]),
         "orc_num_threads": (I32, []),
@@ -212,6 +215,11 @@ def quantize(x: np.ndarray, fmt: int = NVFP4, block: int = 16, g_in=None, e8m0_f
         sc = np.zeros((rows, cols // 32), np.uint8)
         rc = L.orc_quantize_mxfp4_1d_r(_ptr(x), rows, cols, dt, 1 if e8m0_floor else 0, _ptr(codes), _ptr(sc))
         out.update(codes=codes, scales=sc, g=np.float32(1.0))
+    elif fmt == MXFP8 and block == 32:
+        codes = np.zeros((rows, cols), np.uint8)
+        sc = np.zeros((rows, cols // 32), np.uint8)
+        rc = L.orc_quantize_mxfp8_1d(_ptr(x), rows, cols, dt, _ptr(codes), _ptr(sc))
+        out.update(codes=codes, scales=sc, g=np.float32(1.0))
     elif fmt == NVFP4 and block == 256:
         codes = np.zeros((rows, cols // 2), np.uint8)
         sc = np.zeros((rows, cols // 16), np.uint8)
@@ -267,9 +275,15 @@ def swizzle_scales_grouped(rm: np.ndarray, offsets: np.ndarray) -> np.ndarray:
 
 
 def dequantize(codes: np.ndarray, scales_rm: np.ndarray, g: float, fmt: int = NVFP4) -> np.ndarray:
-    """x_hat = E2M1(code) * dec(scale) (* g for NVFP4), in float64, shape [rows, cols]."""
+    """x_hat = E2M1(code) * dec(scale) (* g for NVFP4), or E4M3(code) * dec(scale) for
+    MXFP8 (one code per byte), in float64, shape [rows, cols]."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales_rm = np.ascontiguousarray(scales_rm, dtype=np.uint8)
+    if fmt == MXFP8:
+        rows, cols = codes.shape
+        out = np.zeros((rows, cols), np.float64)
+        _L().orc_dequantize_mxfp8(_ptr(codes), _ptr(scales_rm), rows, cols, _ptr(out))
+        return out
     rows, half = codes.shape
     cols = half * 2
     out = np.zeros((rows, cols), np.float64)

@@ -410,6 +410,54 @@ int orc_quantize_mxfp4_1d_r(const void* x, int64_t rows, int64_t cols, int dtype
 }
 
 /* ------------------------------------------------------------------------- */
+/* MXFP8: E4M3 elements with an E8M0 scale per 32 ([P1] 3.1 names MXFP8 beside     */
+/* MXFP4 in the OCP microscaling family, pure-exponent scales; [P1] 3.4 wants an     */
+/* FP8 operand opposite an FP4 one).  The pages fix no scale rule for it; the       */
+/* reading follows the MXFP4 one: the nearest power of two of amax_b / 448, 448     */
+/* being E4M3's largest value as 6 is E2M1's.  Elements: sign in bit 7, magnitude   */
+/* by the E4M3 encoder above (nearest, ties to the even mantissa, saturating).      */
+/* ------------------------------------------------------------------------- */
+
+static uint8_t mxfp8_encode_block(const float* xs, int n, float amax_b, uint8_t* codes) {
+    uint8_t sb = orc_e8m0_encode(amax_b / 448.0f);
+    float f = (float)ldexp(1.0, 127 - (int)sb);  /* exact scaling, as for MXFP4 */
+    for (int i = 0; i < n; ++i) {
+        float v = xs[i] * f;
+        codes[i] = (uint8_t)((signbit(v) ? 0x80 : 0) | orc_e4m3_encode(fabsf(v)));
+    }
+    return sb;
+}
+
+/* [rows, cols] -> codes [rows, cols] (one byte per element), scales_rm [rows, cols / 32]. */
+int orc_quantize_mxfp8_1d(const void* x, int64_t rows, int64_t cols, int dtype, uint8_t* codes,
+                          uint8_t* scales_rm) {
+    for (int64_t i = 0; i < rows * cols; ++i)
+        if (!isfinite(load_elem(x, i, dtype))) return ORC_ERR_NONFINITE;
+    tables_ready();
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float xs[32];
+        for (int64_t b = 0; b < cols / 32; ++b) {
+            float amax_b = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                xs[i] = load_elem(x, r * cols + b * 32 + i, dtype);
+                if (fabsf(xs[i]) > amax_b) amax_b = fabsf(xs[i]);
+            }
+            scales_rm[r * (cols / 32) + b] = mxfp8_encode_block(xs, 32, amax_b, codes + r * cols + b * 32);
+        }
+    }
+    return ORC_OK;
+}
+
+/* x_hat = E4M3(code) * 2^(scale - 127), in FP64. */
+void orc_dequantize_mxfp8(const uint8_t* codes, const uint8_t* scales_rm, int64_t rows, int64_t cols,
+                          double* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < cols; ++k)
+            out[r * cols + k] = orc_e4m3_decode(codes[r * cols + k]) * orc_e8m0_decode(scales_rm[r * (cols / 32) + k / 32]);
+}
+
+/* ------------------------------------------------------------------------- */
 /* 2-D NVFP4 weight quantize ([P2] training-recipe passage: one scale per 16x16 */
 /* weight patch, so the forward W and the backward W^T share one quantization). */
 /* Emits W's codes and 1x16-expanded scales, and W^T's codes and scales.        */

@@ -13,6 +13,7 @@ import pytest
 import oracle
 import test_oracle_formats as tf
 import test_oracle_gemm as tg
+import test_oracle_mxfp8 as tm
 import test_oracle_next as tn
 import test_oracle_quantize as tq
 
@@ -137,6 +138,18 @@ C_MUTATIONS = [
      "uint8_t sb = floor_mode ? orc_e8m0_encode_floor(amax_b) : orc_e8m0_encode(amax_b / 6.0f);",
      "uint8_t sb = orc_e8m0_encode(amax_b / 6.0f);",
      [tn.test_quantize_mxfp4_floor_block_maximum_codes]),
+    ("MXFP8 scale maps the block amax to 6 instead of 448",
+     "uint8_t sb = orc_e8m0_encode(amax_b / 448.0f);",
+     "uint8_t sb = orc_e8m0_encode(amax_b / 6.0f);",
+     [lambda: tm.test_mxfp8_worked_blocks(0), lambda: tm.test_mxfp8_scale_is_the_nearest_power_of_two_of_amax_over_448(448.0, 127)]),
+    ("MXFP8 drops the element sign",
+     "codes[i] = (uint8_t)((signbit(v) ? 0x80 : 0) | orc_e4m3_encode(fabsf(v)));",
+     "codes[i] = (uint8_t)orc_e4m3_encode(fabsf(v));",
+     [tm.test_mxfp8_sign_symmetry, tm.test_mxfp8_every_e4m3_code_round_trips]),
+    ("MXFP8 dequantize forgets the block scale",
+     "out[r * cols + k] = orc_e4m3_decode(codes[r * cols + k]) * orc_e8m0_decode(scales_rm[r * (cols / 32) + k / 32]);",
+     "out[r * cols + k] = orc_e4m3_decode(codes[r * cols + k]);",
+     [tm.test_mxfp8_error_bound]),
     ("Hadamard butterfly difference reversed",
      "v[j + h] = p - q;",
      "v[j + h] = q - p;",
