@@ -354,6 +354,7 @@ def run_decode(args, dist: Dist, dev):
 
 # ---------------------------------------------------------------- the other configurations
 FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 ratio (4.5 / 2.25 PFLOP/s): the mixed FP4 x FP8 MMA's rate
 MIN_TIMED_S = 0.4   # each sub-workload is timed over at least this long (clock samples cover it)
 MIN_S_OVERRIDE = None  # --min-seconds: one minimum for every timed loop (short runs under a profiler)
 
@@ -863,7 +864,84 @@ def load_peak_table(dev) -> dict:
     return pk
 
 
-MEASURES = {"prefill": measure_prefill, "train": measure_train, "moe": measure_moe, "quantize": measure_quantize}
+def measure_mixed(args, dev, peaks, cpu: bool) -> dict:
+    """The FP4 x FP8 GEMM (next row f4) on the prefill shape 8192^3: BF16 activations
+    quantized to MXFP8 every step (one pass: E8M0 scales need no tensor amax), weights
+    pre-quantized to MXFP4 and rotating past L2, BF16 out.  The MMA runs at the FP8 rate,
+    so the tensor roofline is the measured BF16 peak x 2."""
+    import block_scaled_fp4_04_b200 as fp4
+    m = n = k = 8192
+    x, w = workloads.prefill_inputs(device="cpu")
+    xd = x.to(dev)
+    per_copy = n * k // 2 + fp4.fp4_scales_bytes(n, k, fp4.MXFP4)
+    copies = _copies(per_copy)
+    w_dev = w.to(dev)
+    wq = [fp4.quantize(w_dev, fp4.MXFP4, 32) for _ in range(copies)]
+    del w_dev
+    L = fp4.lib()
+    P = lambda t: t.data_ptr()
+    xc = torch.empty(m, k, dtype=torch.uint8, device=dev)
+    xs = torch.empty(fp4.fp4_scales_bytes(m, k, fp4.MXFP8), dtype=torch.uint8, device=dev)
+    d = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+    sp = torch.cuda.current_stream().cuda_stream
+
+    def quant(src=None):
+        if L.fp4_quantize(P(src if src is not None else xd), m, k, fp4.BF16, fp4.MXFP8, 32, P(xc), P(xs), None, None,
+                          None, None, None, 0, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    def gemm(i):
+        q = wq[i % copies]
+        if L.fp4_gemm_mixed(fp4.MXFP8, P(xc), P(xs), fp4.MXFP4, P(q.codes), P(q.scales), m, n, k, P(d), fp4.BF16, sp):
+            raise RuntimeError(fp4.fp4_last_error())
+
+    def step(i, src=None):
+        quant(src)
+        gemm(i)
+
+    di = dev.index or 0
+    step_ms, batches, clk = timed_batches(step, args.steps, args.warmup, di)
+    gemm_ms, _, gclk = timed_batches(gemm, args.steps, args.warmup, di)
+    _check(fp4)
+    flop = 2.0 * m * n * k
+    fp8_peak = peaks["fp4"] / FP4_PER_BF16 * FP8_PER_BF16
+    achieved = flop / (gemm_ms * 1e-3) / 1e12
+    x_host = x.pin_memory()
+    d_host = torch.empty(m, n, dtype=torch.bfloat16).pin_memory()
+    x_stage = torch.empty_like(xd)
+    e2e_ms = _e2e(lambda i: step(i, x_stage), [x_host], [x_stage], [d_host], [d], args.steps, args.warmup)
+    _check(fp4)
+    rec = {"value": flop / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms,
+           "steps_per_batch": args.steps, "batches": len(batches), "timing": "median over batches",
+           "config": {"workload": "mixed FP4 x FP8 GEMM M=N=K=8192: bf16 activations quantized to MXFP8 every "
+                                  "step, weights MXFP4 pre-quantized, bf16 out",
+                      "step": "fp4_quantize (MXFP8, one pass) + fp4_gemm_mixed (2 launches)",
+                      "l2": f"weights rotate over {copies} pre-quantized copies ({copies * per_copy / 2**20:.0f} MiB)"},
+           "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, mx, 1 acc, kind::mxf8f6f4>",
+                        "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
+                        "peak_source": peaks["fp4_source"].replace(f"x {FP4_PER_BF16:g} (nominal FP4/BF16",
+                                                                   f"x {FP8_PER_BF16:g} (nominal FP8/BF16"),
+                        "launch_ms": gemm_ms, "traffic": traffic_for("mixed_gemm"), "gemm_clocks": gclk},
+           "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                   "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2},
+           "gpu_launches_per_step": 2, "clocks": clk}
+    if cpu:
+        import oracle
+        rows = 8
+        xb = workloads.bf16_bits(x)
+        ow = oracle.quantize(w.numpy(), oracle.MXFP4, 32)
+        w_hat = oracle.dequantize(ow["codes"], ow["scales"], ow["g"], oracle.MXFP4)
+        v, cores, reps = _oracle_rows_gemm_rate(np.ascontiguousarray(xb[:rows]), oracle.MXFP8, 32, w_hat)
+        rec["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{reps} x (MXFP8-quantize {rows} rows of X, FP64 product with the "
+                                         "8192 x 8192 dequantized MXFP4 weights)"}
+    del wq, xd, xc, xs, d, x_stage
+    torch.cuda.empty_cache()
+    return rec
+
+
+MEASURES = {"prefill": measure_prefill, "train": measure_train, "moe": measure_moe, "quantize": measure_quantize,
+            "mixed": measure_mixed}
 
 
 def cpu_baseline_decode(budget_s: float = 12.0):
@@ -943,7 +1021,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "train", "quantize"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "moe", "train", "quantize", "mixed"],
                     help="decode: the headline line, with the other configurations as sub-records; any other "
                          "value prints that configuration's record alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -22,7 +22,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfp4.so")
 
-NVFP4, MXFP4 = 0, 1
+NVFP4, MXFP4, MXFP8 = 0, 1, 2  # MXFP8: E4M3 elements, one byte each (the mixed GEMM's FP8 operand)
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = range(6)
 GEMM_WEIGHTS_READY = 1
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
                 "fp4_gemm": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, P]),
                 "fp4_gemm_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, SZ, ctypes.c_uint, P]),
                 "fp4_gemm_noalloc": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
+                "fp4_gemm_mixed": (I32, [I32, P, P, I32, P, P, I64, I64, I64, P, I32, P]),
                 "fp4_gemm_epilogue_workspace_size": (SZ, [I64, I64, I64, I32, I32]),
                 "fp4_gemm_epilogue": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, I32, P, I32, P, P, P, P, P,
                                             SZ, P]),
@@ -228,6 +229,11 @@ def fp4_gemm_noalloc(fmt, A, sA, gA, B, sB, gB, M, N, K, D, out_dtype, stream=No
                                   _s(stream)))
 
 
+def fp4_gemm_mixed(a_fmt, A, sA, b_fmt, B, sB, M, N, K, D, out_dtype, stream=None):
+    """D = A B^T with A and B each MXFP4 or MXFP8 (the FP4 x FP8 GEMM)."""
+    _check(lib().fp4_gemm_mixed(a_fmt, _p(A), _p(sA), b_fmt, _p(B), _p(sB), M, N, K, _p(D), out_dtype, _s(stream)))
+
+
 def fp4_gemm_grouped(fmt, num_groups, offsets, A, sA, gA, B, sB, gB, total_rows, N, K, D, out_dtype,
                      workspace=None, workspace_bytes=0, stream=None):
     _check(lib().fp4_gemm_grouped(fmt, num_groups, _p(offsets), _p(A), _p(sA), _p(gA), _p(B), _p(sB), _p(gB),
@@ -287,7 +293,7 @@ def quantize(x: torch.Tensor, fmt: int = NVFP4, block: Optional[int] = None, glo
     x = x.contiguous()
     rows, cols = (1, x.numel()) if x.dim() == 1 else tuple(x.shape)
     dev = x.device
-    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    codes = torch.empty(rows, cols if fmt == MXFP8 else cols // 2, dtype=torch.uint8, device=dev)
     scales = torch.empty(fp4_scales_bytes(rows, cols, fmt), dtype=torch.uint8, device=dev)
     g = torch.empty(1, dtype=torch.float32, device=dev)
     codesT = scalesT = None
@@ -312,6 +318,18 @@ def gemm(a: Quantized, b: Quantized, out_dtype=torch.bfloat16, workspace: Option
     ws = (workspace or Workspace(a.codes.device)).get(nbytes) if nbytes else None
     fp4_gemm(a.fmt, a.codes, a.scales, a.g, b.codes, b.scales, b.g, M, N, K, out, oc, ws,
              ws.numel() if ws is not None else 0, stream)
+    return out
+
+
+def gemm_mixed(a: Quantized, b: Quantized, out_dtype=torch.bfloat16, stream=None,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """D[M, N] = A . B^T for A and B each quantized as MXFP4 or MXFP8 (K % 128 == 0)."""
+    assert a.cols == b.cols
+    M, N, K = a.rows, b.rows, a.cols
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+    oc = BF16 if out.dtype == torch.bfloat16 else F32
+    fp4_gemm_mixed(a.fmt, a.codes, a.scales, b.fmt, b.codes, b.scales, M, N, K, out, oc, stream)
     return out
 
 

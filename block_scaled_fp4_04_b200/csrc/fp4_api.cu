@@ -84,7 +84,7 @@ const char* fp4_last_error(void) { return g_err; }
 
 size_t fp4_scales_bytes(int64_t rows, int64_t cols, fp4_fmt fmt) {
   if (rows <= 0 || cols <= 0) return 0;
-  const int64_t blk = fmt == FP4_MXFP4 ? 32 : 16;
+  const int64_t blk = fmt == FP4_MXFP4 || fmt == FP4_MXFP8 ? 32 : 16;
   const int64_t scols = (cols + blk - 1) / blk;
   return static_cast<size_t>(((rows + 127) / 128) * 128 * ((scols + 3) / 4) * 4);
 }
@@ -122,7 +122,13 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   if (rows <= 0 || cols <= 0) return fail(FP4_ERR_INVALID_ARG, "rows and cols must be positive");
   if (cols % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "cols must be a multiple of 32");
   if (in_dtype != FP4_F32 && in_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "in_dtype");
-  if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4) return fail(FP4_ERR_INVALID_ARG, "fmt");
+  if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4 && fmt != FP4_MXFP8) return fail(FP4_ERR_INVALID_ARG, "fmt");
+  if (fmt == FP4_MXFP8) {
+    if (block != 32) return fail(FP4_ERR_INVALID_ARG, "MXFP8 block must be 32");
+    if (num_groups) return fail(FP4_ERR_UNSUPPORTED, "grouped MXFP8 quantization");
+    if (variant != kQuantPlain) return fail(FP4_ERR_UNSUPPORTED, "quantizer variants are FP4 only");
+    variant = kQuantFp8;
+  }
   const bool two_d = block == 256;
   if (fmt == FP4_NVFP4 && block != 16 && block != 256) return fail(FP4_ERR_INVALID_ARG, "NVFP4 block must be 16 or 256");
   if (fmt == FP4_MXFP4 && block != 32) return fail(FP4_ERR_INVALID_ARG, "MXFP4 block must be 32");
@@ -147,7 +153,7 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   if (s != FP4_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bf16 = in_dtype == FP4_BF16;
-  const int mx = fmt == FP4_MXFP4;
+  const int mx = fmt == FP4_MXFP4 || fmt == FP4_MXFP8;
   cudaError_t e = cudaSuccess;
   if (variant == kQuantPlain && !two_d && !num_groups && quantize_small_fits(rows, cols, bf16, mx)) {
     // one launch: amax, global scale and encode by one thread-block cluster
@@ -228,7 +234,7 @@ fp4_status fp4_quantize_grouped(const void* x, int64_t rows, int64_t cols, fp4_d
                                 float* global_out, const float* global_in, void* workspace,
                                 size_t workspace_bytes, void* stream) {
   if (num_groups <= 0) return fail(FP4_ERR_INVALID_ARG, "num_groups must be positive");
-  return quantize_common(x, rows, cols, in_dtype, fmt, fmt == FP4_MXFP4 ? 32 : 16, codes_out, scales_out,
+  return quantize_common(x, rows, cols, in_dtype, fmt, fmt == FP4_NVFP4 ? 16 : 32, codes_out, scales_out,
                          global_out, nullptr, nullptr, global_in, workspace, workspace_bytes, num_groups, offsets,
                          stream);
 }
@@ -266,6 +272,43 @@ static fp4_status gemm_common(const GemmProblem& g, fp4_fmt fmt, fp4_dtype out_d
   const char* why = nullptr;
   cudaError_t err = cudaSuccess;
   const int rc = launch_gemm(g, status, static_cast<cudaStream_t>(stream), &why, &err);
+  if (rc == 1) return fail(FP4_ERR_INVALID_ARG, why);
+  if (rc == 2) return cuda_fail(err, "gemm launch");
+  return FP4_OK;
+}
+
+static bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
+
+fp4_status fp4_gemm_mixed(fp4_fmt a_fmt, const uint8_t* A, const uint8_t* sA, fp4_fmt b_fmt, const uint8_t* B,
+                          const uint8_t* sB, int64_t M, int64_t N, int64_t K, void* D, fp4_dtype out_dtype,
+                          void* stream) {
+  if ((a_fmt != FP4_MXFP4 && a_fmt != FP4_MXFP8) || (b_fmt != FP4_MXFP4 && b_fmt != FP4_MXFP8))
+    return fail(FP4_ERR_INVALID_ARG, "a_fmt and b_fmt must each be FP4_MXFP4 or FP4_MXFP8");
+  if (out_dtype != FP4_F32 && out_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "out_dtype");
+  if (!A || !B || !sA || !sB || !D) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (M <= 0 || N <= 0 || K <= 0) return fail(FP4_ERR_INVALID_ARG, "M, N, K must be positive");
+  if (K % 128 != 0) return fail(FP4_ERR_INVALID_ARG, "K must be a multiple of 128");
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256) return fail(FP4_ERR_UNSUPPORTED, "dimension too large");
+  if (!aligned32(A) || !aligned32(B) || !aligned16(sA) || !aligned16(sB) || !aligned16(D))
+    return fail(FP4_ERR_INVALID_ARG, "A and B must be 32-byte aligned, scales and D 16-byte aligned");
+  unsigned* status;
+  fp4_status s = device_state(&status);
+  if (s != FP4_OK) return s;
+  GemmProblem g{};
+  g.mx = 1;
+  g.A = A;
+  g.sA = sA;
+  g.B = B;
+  g.sB = sB;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.D = D;
+  g.out_bf16 = out_dtype == FP4_BF16;
+  const char* why = nullptr;
+  cudaError_t err = cudaSuccess;
+  const int rc = launch_gemm_mixed(g, a_fmt == FP4_MXFP8, b_fmt == FP4_MXFP8, status, static_cast<cudaStream_t>(stream),
+                                   &why, &err);
   if (rc == 1) return fail(FP4_ERR_INVALID_ARG, why);
   if (rc == 2) return cuda_fail(err, "gemm launch");
   return FP4_OK;

@@ -84,6 +84,15 @@ __device__ __forceinline__ uint32_t e4m3_code(float r) {
   return d & 0xFFu;
 }
 
+// Four scaled values to four E4M3 bytes, the first in the low byte: hardware nearest-even
+// conversion that saturates at +-448 and keeps the sign of zero.
+__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
 // Exact value of an E4M3 code (< 0x7F): subnormal m * 2^-9, else (1 + m/8) * 2^(e-7).
 __device__ __forceinline__ float e4m3_value(uint32_t c) {
   const uint32_t e = (c >> 3) & 15u, m = c & 7u;

@@ -92,6 +92,7 @@ struct GemmArgs {
   const float* q_g;    // global scale of the NVFP4 result (device)
   int64_t q_atoms;     // scale atoms per 128-row block of the result: ceil(N/16, 4) / 4
   unsigned* amax_out;  // max |result| as float bits (zeroed before the launch), or null
+  uint32_t f8_fmt;     // kind::mxf8f6f4: A's format | B's format << 3 (E4M3 0, E2M1 5)
 };
 
 struct Work {
@@ -223,8 +224,11 @@ struct Sched {
 template <int BN>
 constexpr int pipes_per_cta() { return BN <= 32 ? FP4_SMALL_N_PIPES : BN <= 64 ? 2 : 1; }
 
-template <int BN, bool MX, int ACC, bool PAIR = false>
+// F8: the kind::mxf8f6f4 MMA (E2M1 or E4M3 operands, one byte per element in shared
+// memory, an E8M0 scale per 32): a stage holds 128 K elements, one scale atom per row-block.
+template <int BN, bool MX, int ACC, bool PAIR = false, bool F8 = false>
 struct Cfg {
+  static_assert(!F8 || (MX && !PAIR), "mixed-format MMAs: E8M0 scales, single-CTA tiles");
   static_assert(!PAIR || (BN == 256 && ACC == 1), "CTA pairs run 256 x 256 tiles");
   static constexpr int kP = pipes_per_cta<BN>();
   // Single-pipeline kernels (128/256-wide tiles) add copier warps that move each stage's
@@ -238,13 +242,15 @@ struct Cfg {
   static constexpr int kEpiWarps = kSepCp ? 8 : 4;
   static constexpr int kEpiCols = BN * 4 / kEpiWarps;  // accumulator columns per epilogue thread
   static constexpr int kThreads = kSepCp ? 64 + 32 * kEpiWarps + 32 * kCopiers : 192 * kP;
-  static constexpr int kAtomsKT = MX ? 2 : 4;           // scale atoms per 256-wide K step
+  static constexpr int kAtomsKT = F8 ? 1 : MX ? 2 : 4;  // scale atoms per stage (256 K; 128 K for F8)
   static constexpr int kNRB = BN >= 128 ? BN / 128 : 1;  // B scale row-blocks per tile
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * 128;  // a pair's CTA holds half of B's rows
   static constexpr int kSFABytes = kAtomsKT * 512;
   static constexpr int kSFBBytes = kNRB * kAtomsKT * 512;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // a multiple of 1024
+  // rounded up to 1024 bytes (the 128-byte swizzle's alignment): only the mixed-format
+  // stages (one scale atom per row-block) need the padding
+  static constexpr int kStageBytes = (kABytes + kBBytes + kSFABytes + kSFBBytes + 1023) / 1024 * 1024;
   // grouped schedules use 128-wide tiles only, so multi-pipeline kernels skip the group tables
   static constexpr int kGroupBytes = kP == 1 ? (PAIR ? 3 : 2) * (kMaxGroups + 1) * 4 : 0;
   static constexpr int kMiscBytes = 1024 /*barriers, flags*/ + kGroupBytes;
@@ -397,12 +403,12 @@ __device__ __forceinline__ void epi_sync(int sub, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + sub), "r"(nthreads) : "memory");
 }
 
-template <int BN, bool MX, int ACC, bool PAIR>
-__global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
+template <int BN, bool MX, int ACC, bool PAIR, bool F8 = false>
+__global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR, F8>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const GemmArgs p) {
-  using C = Cfg<BN, MX, ACC, PAIR>;
+  using C = Cfg<BN, MX, ACC, PAIR, F8>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
@@ -696,10 +702,21 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
             copy_stage_sf(st, sfa_t, kb);
           }
           ++nstage;
-          const int krem = p.K - kb * 256;
-          const int nk = krem >= 256 ? 4 : (krem + 63) / 64;
+          const int krem = p.K - kb * (F8 ? 128 : 256);
+          const int nk = F8 ? (krem >= 128 ? 4 : (krem + 31) / 32) : (krem >= 256 ? 4 : (krem + 63) / 64);
           const uint64_t adesc = smem_desc_sw128(st);
           const uint64_t bdesc = smem_desc_sw128(st + C::kABytes);
+          if constexpr (F8) {
+            // four K = 32 MMAs over the stage's 128-byte rows (one byte per element of
+            // either format); MMA k reads byte k of each row's 32-bit scale word
+            for (int k = 0; k < nk; ++k) {
+              const uint32_t sfid = static_cast<uint32_t>(k);
+              const uint32_t idesc = mma_idesc_f8(BN, p.f8_fmt & 7u, (p.f8_fmt >> 3) & 7u, sfid, sfid, kMTile);
+              const uint32_t accum = (kb > w.kb0 || k > 0) ? 1u : 0u;
+              tc_mma_mxf8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t | (sfid << 30), sfb_t | (sfid << 30),
+                              accum);
+            }
+          } else {
           for (int k = 0; k < nk; ++k) {
             const uint32_t a_idx = MX ? (k >> 1) : k;
             const uint32_t sfid = MX ? (k & 1) * 2 : 0;
@@ -715,6 +732,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR>::kThreads, 1)
               tc_mma_mxfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
             else
               tc_mma_nvfp4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, ta, tb, accum);
+          }
           }
           if constexpr (PAIR)
             tc_commit_pair_mc(&empty[stage], 3);  // frees the stage in both CTAs
@@ -1036,6 +1054,23 @@ static bool encode_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, k] E2M1 codes, packed two per byte in global memory (row pitch k / 2 bytes),
+// copied into shared memory one byte per element: each 16 codes (8 bytes) followed by an
+// 8-byte gap, the operand layout of the kind::mxf8f6f4 MMA.  CUDA's documented limits for
+// this data type: a 32-byte aligned base, k a multiple of 128, a row pitch that is a
+// multiple of 32 bytes, and boxes 128 elements wide.
+static bool encode_map_u4(CUtensorMap* m, const void* base, uint64_t k, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {k, rows};
+  const cuuint64_t strides[1] = {k / 2};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Small host cache of encoded tensor maps keyed by (address, shape, box): decode-style
 // callers pass the same buffers every step, and encoding costs host time on every call.
 // A map only describes addresses, so a stale entry is just another valid encoding.
@@ -1202,11 +1237,11 @@ size_t gemm_bf16a_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return (kQuantWorkspaceBytes + 255) / 256 * 256 + gemm_workspace_bytes(M, N, K, 0);
 }
 
-template <int BN, bool MX, int ACC, bool PAIR>
+template <int BN, bool MX, int ACC, bool PAIR, bool F8 = false>
 static cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
                        const GemmArgs& a, int64_t units, cudaStream_t st) {
-  using C = Cfg<BN, MX, ACC, PAIR>;
-  auto kern = fp4_gemm_kernel<BN, MX, ACC, PAIR>;
+  using C = Cfg<BN, MX, ACC, PAIR, F8>;
+  auto kern = fp4_gemm_kernel<BN, MX, ACC, PAIR, F8>;
   // the shared-memory opt-in is per device; set it once per (kernel, device)
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -1379,6 +1414,58 @@ int launch_gemm(const GemmProblem& g, unsigned* status, cudaStream_t st, const c
     a.sfb_rbs = static_cast<int>((rowsB + 127) / 128);
   }
   const cudaError_t e = g.mx ? dispatch<true>(pl, ta, tb, tsa, tsb, a, st) : dispatch<false>(pl, ta, tb, tsa, tsb, a, st);
+  if (e != cudaSuccess) {
+    *err = e;
+    return 2;
+  }
+  return 0;
+}
+
+// FP4 x FP8 ("Rubin FP4 GEMM overview" 3.4: an FP4 operand opposite an FP8 one): A and
+// B each MXFP4 or MXFP8, D = A B^T on kind::mxf8f6f4 MMAs.  Dense, whole tiles on single
+// CTAs; K a multiple of 128.
+int launch_gemm_mixed(const GemmProblem& g, int a_fp8, int b_fp8, unsigned* status, cudaStream_t st,
+                      const char** why, cudaError_t* err) {
+  const int sms = num_sms();
+  const int64_t tiles256 = ((g.M + 127) / 128) * ((g.N + 255) / 256);
+  const int BN = (g.N >= 256 && tiles256 >= sms) ? 256 : 128;
+  CUtensorMap ta, tb;
+  const bool ok_a = a_fp8 ? make_tensor_map_u8(&ta, g.A, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M), 128)
+                          : encode_map_u4(&ta, g.A, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M), 128);
+  const bool ok_b = b_fp8 ? make_tensor_map_u8(&tb, g.B, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N),
+                                               static_cast<uint32_t>(BN))
+                          : encode_map_u4(&tb, g.B, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N),
+                                          static_cast<uint32_t>(BN));
+  if (!ok_a || !ok_b) {
+    *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
+    return 1;
+  }
+  const int64_t atoms_k = g.K / 128;  // one E8M0 per 32 K elements, four per atom row
+  GemmArgs a{};
+  a.sfa = g.sA;
+  a.sfb = g.sB;
+  a.sfa_rb_bytes = atoms_k * 512;
+  a.sfb_rb_bytes = atoms_k * 512;
+  a.sf_atoms_k = static_cast<int>(atoms_k);
+  a.sfb_rbs = static_cast<int>((g.N + 127) / 128);
+  a.Mk = static_cast<int>(g.M);
+  a.Nk = static_cast<int>(g.N);
+  a.K = static_cast<int>(g.K);
+  a.num_kb = static_cast<int>(g.K / 128);
+  a.out = g.D;
+  a.out_bf16 = g.out_bf16;
+  a.ldo = g.N;
+  const int esz = g.out_bf16 ? 2 : 4;
+  a.vec_store = ((g.N * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(g.D) & 15) == 0) ? 1 : 0;
+  a.mode = kModeTile;
+  a.tiles_m = static_cast<int>((g.M + 127) / 128);
+  a.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
+  a.group_m = 16;
+  a.total_units = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+  a.status = status;
+  a.f8_fmt = (a_fp8 ? kFmtE4M3 : kFmtE2M1) | ((b_fp8 ? kFmtE4M3 : kFmtE2M1) << 3);
+  const cudaError_t e = BN == 256 ? run<256, true, 1, false, true>(ta, tb, ta, tb, a, a.total_units, st)
+                                  : run<128, true, 2, false, true>(ta, tb, ta, tb, a, a.total_units, st);
   if (e != cudaSuccess) {
     *err = e;
     return 2;

@@ -26,7 +26,7 @@ int num_sms();  // SM count of the current device (cached per device)
 cudaError_t launch_amax(const void* x, int64_t n, int bf16, uint32_t* ws, float* amax_out, float* g_out,
                         unsigned* status, cudaStream_t st, int rht = 0, uint32_t signs = 0);
 // Quantizer variants of the 1-D kernel (see fp4_quantize.cu).
-enum { kQuantPlain = 0, kQuantMxFloor = 1, kQuantSR = 2, kQuantRHT = 3 };
+enum { kQuantPlain = 0, kQuantMxFloor = 1, kQuantSR = 2, kQuantRHT = 3, kQuantFp8 = 4 };
 cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf16, int mx, uint8_t* codes,
                                uint8_t* scales, const float* g, const int32_t* offsets, int num_groups,
                                unsigned* status, cudaStream_t st, int variant = kQuantPlain,
@@ -107,5 +107,10 @@ int launch_decode(const DecodeProblem& q, unsigned* status, cudaStream_t st, con
 // Returns 0 on success, 1 on an unsupported shape / too-small workspace (message in
 // *why), or 2 on a CUDA error (code in *err).
 int launch_gemm(const GemmProblem& p, unsigned* status, cudaStream_t st, const char** why, cudaError_t* err);
+// D = A B^T with A and B each MXFP4 (a_fp8 / b_fp8 = 0) or MXFP8 (1), kind::mxf8f6f4 MMAs;
+// K % 128 == 0, A and B 32-byte aligned.  Uses g.A, g.sA, g.B, g.sB, g.M, g.N, g.K, g.D,
+// g.out_bf16.
+int launch_gemm_mixed(const GemmProblem& g, int a_fp8, int b_fp8, unsigned* status, cudaStream_t st,
+                      const char** why, cudaError_t* err);
 
 }  // namespace fp4

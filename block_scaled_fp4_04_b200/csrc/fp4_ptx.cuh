@@ -196,6 +196,21 @@ __device__ __forceinline__ void tc_mma_mxfp4(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 
+// D (+)= A * B^T with an E8M0 scale per 32 K elements of each operand; A and B each E2M1
+// or E4M3 (formats in the instruction descriptor), K = 32 per instruction.  An E2M1
+// operand sits in shared memory one byte per element (16 codes in 8 bytes, then 8 bytes
+// of gap: the layout a CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B tensor copy writes).
+__device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+      "}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ CTA pairs
 // A cluster of two CTAs on neighbouring SMs that share one MMA of M = 256 rows: CTA
 // rank 0 (the leader) issues every tcgen05 operation for both; operand tiles, scale
@@ -353,6 +368,24 @@ __host__ __device__ __forceinline__ uint32_t mma_idesc(int n, bool mx, uint32_t 
   d |= (static_cast<uint32_t>(n) >> 3) << 17;     // N / 8
   d |= (mx ? 1u : 0u) << 23;                      // scale type
   d |= (static_cast<uint32_t>(m) >> 4) << 24;     // M / 16
+  d |= (a_sf_id & 3u) << 29;
+  return d;
+}
+
+// Instruction descriptor of the kind::mxf8f6f4 block-scaled MMA: operand formats
+// (E4M3 = 0, E2M1 = 5) in bits 7..9 (A) and 10..12 (B), N / 8, E8M0 scales, M / 16,
+// K = 32 (bit 31 clear), and the byte of each operand's 32-bit scale word the
+// instruction reads (one E8M0 per row per 32 K elements).
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+__host__ __device__ __forceinline__ uint32_t mma_idesc_f8(int n, uint32_t a_fmt, uint32_t b_fmt, uint32_t a_sf_id,
+                                                          uint32_t b_sf_id, int m = 128) {
+  uint32_t d = 0;
+  d |= (b_sf_id & 3u) << 4;
+  d |= (a_fmt & 7u) << 7;
+  d |= (b_fmt & 7u) << 10;
+  d |= (static_cast<uint32_t>(n) >> 3) << 17;
+  d |= 1u << 23;  // E8M0 scales
+  d |= (static_cast<uint32_t>(m) >> 4) << 24;
   d |= (a_sf_id & 3u) << 29;
   return d;
 }

@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int UPT = 2;                                        // blocks per thread per tile
   static_assert(VAR != kQuantMxFloor || MX, "the rounded-down scale is an E8M0 one");
   static_assert(VAR != kQuantSR || (!MX && BLOCK == 16), "stochastic rounding: NVFP4");
+  static_assert(VAR != kQuantFp8 || (MX && BLOCK == 32), "MXFP8: E4M3 elements in 32-blocks");
   constexpr int RW = VAR == kQuantSR ? BLOCK / 4 : 0;  // 16-byte loads of random words per block
 
   __shared__ int s_rb[kMaxGroups + 1];
@@ -423,12 +424,28 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       uint32_t sb;
       float mul;
       if constexpr (MX) {
-        sb = VAR == kQuantMxFloor ? e8m0_floor_code(amax_b) : e8m0_code(__fdiv_rn(amax_b, 6.0f));
+        // MXFP4: nearest power of two of amax_b / 6 (or rounded down); MXFP8: of amax_b / 448,
+        // E4M3's largest value
+        sb = VAR == kQuantMxFloor ? e8m0_floor_code(amax_b)
+                                  : e8m0_code(__fdiv_rn(amax_b, VAR == kQuantFp8 ? 448.0f : 6.0f));
         mul = e8m0_inverse(sb);
       } else {
         mul = nvfp4_block_scale(amax_b, g, sb);
       }
       const bool inf_mul = !MX && isinf(mul);  // 1/denom overflowed: zeros stay zeros, not NaN
+      if constexpr (VAR == kQuantFp8) {
+        // one E4M3 byte per element: 32 bytes per block, two 16-byte stores
+        uint32_t w8[BLOCK / 4];
+#pragma unroll
+        for (int o = 0; o < BLOCK / 4; ++o)
+          w8[o] = pack4_e4m3(__fmul_rn(v[4 * o], mul), __fmul_rn(v[4 * o + 1], mul), __fmul_rn(v[4 * o + 2], mul),
+                             __fmul_rn(v[4 * o + 3], mul));
+        if (ok[i]) {
+          uint4* dst = reinterpret_cast<uint4*>(p.codes + r * p.cols + bcol * BLOCK);
+          dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+          dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+        }
+      } else {
       uint32_t packed[BLOCK / 8];
 #pragma unroll
       for (int o = 0; o < BLOCK / 8; ++o) {
@@ -461,6 +478,7 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
         uint8_t* dst = p.codes + r * half_cols + bcol * (BLOCK / 2);
         if constexpr (BLOCK == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
       }
       // the scale byte at its place in the atom (rows and blocks past the tensor: 0)
       atom[(rl & 31) * 16 + (rl >> 5) * 4 + bc] = ok[i] ? static_cast<uint8_t>(sb) : 0;
@@ -860,6 +878,9 @@ cudaError_t launch_quantize_1d(const void* x, int64_t rows, int64_t cols, int bf
     case kQuantSR:
       if (mx) return cudaErrorInvalidValue;
       return bf16 ? launch_q1d_t<BF, 16, false, kQuantSR>(a, st) : launch_q1d_t<float, 16, false, kQuantSR>(a, st);
+    case kQuantFp8:
+      if (!mx) return cudaErrorInvalidValue;
+      return bf16 ? launch_q1d_t<BF, 32, true, kQuantFp8>(a, st) : launch_q1d_t<float, 32, true, kQuantFp8>(a, st);
     case kQuantRHT:
       if (bf16)
         return mx ? launch_q1d_t<BF, 32, true, kQuantRHT>(a, st) : launch_q1d_t<BF, 16, false, kQuantRHT>(a, st);

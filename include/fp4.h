@@ -54,7 +54,10 @@
 extern "C" {
 #endif
 
-typedef enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1 } fp4_fmt;
+/* FP4_MXFP8: E4M3 elements (one byte each) with an E8M0 scale per 32 -- the FP8 operand of
+ * fp4_gemm_mixed ("Rubin FP4 GEMM overview" 3.4: an FP4 operand opposite an FP8 one; 3.1
+ * names MXFP8 beside MXFP4 among the OCP microscaling formats). */
+typedef enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1, FP4_MXFP8 = 2 } fp4_fmt;
 typedef enum { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
 typedef enum {
   FP4_OK = 0,
@@ -93,8 +96,10 @@ fp4_status fp4_amax(const void* x_dev, int64_t n, fp4_dtype in_dtype, float* ama
  * round to the nearest E2M1 grid point, ties to the even mantissa; packed two per byte).
  *   fmt/block: (FP4_NVFP4, 16) 1-D blocks along cols; (FP4_MXFP4, 32) 1-D blocks;
  *              (FP4_NVFP4, 256) 16x16 2-D blocks for weights ("MXFP4 / NVFP4 video
- *              transcript", training-recipe passage: W and W^T share one quantization).
- *   codes_out_dev  [rows, cols/2]; scales_out_dev fp4_scales_bytes(rows, cols, fmt).
+ *              transcript", training-recipe passage: W and W^T share one quantization);
+ *              (FP4_MXFP8, 32) E4M3 elements in 1-D blocks (not grouped).
+ *   codes_out_dev  [rows, cols/2] ([rows, cols] for MXFP8); scales_out_dev
+ *              fp4_scales_bytes(rows, cols, fmt).
  *   global_out_dev 1 float: g (NVFP4) or 1.0 (MXFP4).  May be NULL for MXFP4.
  *   codesT_out_dev / scalesT_out_dev: block 256 only -- W^T's codes [cols, rows/2] and
  *              scales fp4_scales_bytes(cols, rows, NVFP4); NULL otherwise.
@@ -103,7 +108,9 @@ fp4_status fp4_amax(const void* x_dev, int64_t n, fp4_dtype in_dtype, float* ama
  * Requires cols % 32 == 0, rows >= 1; block 256 also rows % 32 == 0; x, codes and
  * scales 16-byte aligned.  NVFP4 block scale: sb = E4M3_rn_sat((amax_b / 6) / g);
  * elements x * (1 / (dec(sb) * g)) in FP32.  MXFP4: sb = E8M0 nearest power of two of
- * amax_b / 6 (a midpoint goes up); elements x * 2^(127 - sb). */
+ * amax_b / 6 (a midpoint goes up); elements x * 2^(127 - sb).  MXFP8: sb = E8M0 nearest
+ * power of two of amax_b / 448 (the pages fix no rule for MXFP8; 448 is E4M3's largest
+ * value as 6 is E2M1's); elements E4M3_rn_sat(x * 2^(127 - sb)), sign in bit 7. */
 fp4_status fp4_quantize(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype,
                         fp4_fmt fmt, int block, uint8_t* codes_out_dev, uint8_t* scales_out_dev,
                         float* global_out_dev, uint8_t* codesT_out_dev, uint8_t* scalesT_out_dev,
@@ -228,6 +235,20 @@ fp4_status fp4_gemm_ex(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev,
  * workspace: fp4_gemm_epilogue_workspace_size(M, N, K, fmt, rows_in_place) bytes with
  * rows_in_place = (Dcodes_dev != NULL || amax_out_dev != NULL), zero-filled before first
  * use (left zero-filled).  Plain (not grouped) problems only. */
+/* Mixed-format GEMM ("Rubin FP4 GEMM overview" 3.4: weights in FP4 where they tolerate it,
+ * activations kept in FP8, or the other way round): D[M, N] = A[M, K] B[N, K]^T with each
+ * operand FP4_MXFP4 (E2M1 codes [rows, K/2], E8M0 scales per 32) or FP4_MXFP8 (E4M3
+ * codes [rows, K], E8M0 scales per 32), as fp4_quantize writes them; scales in the
+ * swizzled layout, fp4_scales_bytes(rows, K, fmt) bytes.  FP32 accumulation of the
+ * block-scaled products on the tensor cores (tcgen05 kind::mxf8f6f4: an FP4 operand is
+ * widened to one byte per element in shared memory by the tensor copy).  D row-major,
+ * FP32 or BF16.  Requires K % 128 == 0 (the limit of CUDA's 4-bit tensor-copy type), A
+ * and B 32-byte aligned, scales and D 16-byte aligned; no workspace.  Errors:
+ * FP4_ERR_INVALID_ARG before any launch. */
+fp4_status fp4_gemm_mixed(fp4_fmt a_fmt, const uint8_t* A_dev, const uint8_t* sA_dev, fp4_fmt b_fmt,
+                          const uint8_t* B_dev, const uint8_t* sB_dev, int64_t M, int64_t N, int64_t K,
+                          void* D_dev, fp4_dtype out_dtype, void* stream);
+
 typedef enum { FP4_ACT_NONE = 0, FP4_ACT_RELU = 1 } fp4_act;
 size_t fp4_gemm_epilogue_workspace_size(int64_t M, int64_t N, int64_t K, fp4_fmt fmt, int rows_in_place);
 fp4_status fp4_gemm_epilogue(fp4_fmt fmt, const uint8_t* A_dev, const uint8_t* sA_dev, const float* gA_dev,

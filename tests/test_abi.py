@@ -100,6 +100,36 @@ def test_gemm_rejects_bad_arguments():
                               None, 0, None) == fp4.ERR_INVALID_ARG   # no offsets
 
 
+def test_mixed_gemm_rejects_bad_arguments():
+    L = fp4.lib()
+    good = [fp4.MXFP4, 32, 16, fp4.MXFP8, 64, 16, 128, 128, 256, 16, fp4.BF16, None]
+
+    def call(i, v):
+        a = list(good)
+        a[i] = v
+        return L.fp4_gemm_mixed(*a)
+
+    assert call(0, fp4.NVFP4) == fp4.ERR_INVALID_ARG     # NVFP4 operands use fp4_gemm
+    assert call(3, 7) == fp4.ERR_INVALID_ARG             # b_fmt
+    assert call(8, 192) == fp4.ERR_INVALID_ARG           # K % 128
+    assert call(1, 16) == fp4.ERR_INVALID_ARG            # A only 16-byte aligned
+    assert call(4, 48) == fp4.ERR_INVALID_ARG            # B only 16-byte aligned
+    assert call(9, None) == fp4.ERR_INVALID_ARG          # null D
+    assert call(10, 3) == fp4.ERR_INVALID_ARG            # out dtype
+    assert call(6, 0) == fp4.ERR_INVALID_ARG             # M
+
+
+def test_mxfp8_quantize_arguments():
+    assert fp4.fp4_scales_bytes(300, 1024, fp4.MXFP8) == fp4.fp4_scales_bytes(300, 1024, fp4.MXFP4)
+    assert _rc_quantize(fmt=fp4.MXFP8, block=16) == fp4.ERR_INVALID_ARG
+    assert _rc_quantize(fmt=fp4.MXFP8, block=256) == fp4.ERR_INVALID_ARG
+    L = fp4.lib()
+    assert L.fp4_quantize_grouped(16, 64, 64, fp4.F32, fp4.MXFP8, 2, 16, 16, 16, None, None, 16, 1 << 20, None) \
+        == fp4.ERR_UNSUPPORTED
+    assert L.fp4_quantize_ex(16, 4, 64, fp4.F32, fp4.MXFP8, 32, fp4.QUANT_E8M0_FLOOR, 16, 16, 16, None, None,
+                             None, 16, 1 << 20, None) == fp4.ERR_UNSUPPORTED
+
+
 def test_gemm_ex_rejects_unknown_flags():
     L = fp4.lib()
     assert L.fp4_gemm_ex(fp4.NVFP4, 16, 16, 16, 16, 16, 16, 128, 128, 256, 16, fp4.BF16, None, 0, 6, None) \
