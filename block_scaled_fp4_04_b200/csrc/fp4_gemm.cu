@@ -618,6 +618,12 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR, F8>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
       bool ok = true;
+      // operand bytes a stage's tensor copies complete: a 4-bit operand of the mixed-format
+      // MMA counts its packed bytes (half its footprint in shared memory)
+      uint32_t ab_tx = C::kABytes + C::kBBytes;
+      if constexpr (F8)
+        ab_tx = ((p.f8_fmt & 7u) == kFmtE2M1 ? C::kABytes / 2 : C::kABytes) +
+                (((p.f8_fmt >> 3) & 7u) == kFmtE2M1 ? C::kBBytes / 2 : C::kBBytes);
       while (ok && sch.next(w)) {
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort)) {
@@ -632,7 +638,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR, F8>::kThreads, 1)
             }
           } else if constexpr (C::kSepCp) {
             mbar_arrive_expect_tx(&sf_landed[stage], stage_sf_bytes(w, kb));
-            mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes);
+            mbar_arrive_expect_tx(&full[stage], ab_tx);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + stage_sf_bytes(w, kb));
           }
