@@ -10,6 +10,7 @@ and the last, every column.
   quantization, X and dY quantized with 16-element blocks.
 - MoE: 32 experts, 4096 tokens routed top-4 (16384 rows), K = 2880, N = 5760, MXFP4:
   every expert's sampled rows (16 random plus its first and last).
+- mixed FP4 x FP8: the prefill X quantized to MXFP8 against MXFP4 weights, 8192^3.
 The oracle computes global scales over the whole tensors and quantizes only the rows it
 needs (1-D blocks are independent per row)."""
 import numpy as np
@@ -134,3 +135,24 @@ def test_moe_32_experts_16384_rows_mxfp4():
         ob = oracle.quantize(w[e].numpy(), fp4.MXFP4, 32)
         b_hat = oracle.dequantize(ob["codes"], ob["scales"], ob["g"], fp4.MXFP4)
         _check_rows(D, lo + local, a_hat, b_hat, f"expert {e}")
+
+
+def test_mixed_fp4_fp8_8192_cubed():
+    """The mixed record's configuration: X [8192, 8192] BF16 quantized to MXFP8, W [8192,
+    8192] to MXFP4, D = X W^T through fp4_gemm_mixed; X's codes and scales bit-exact on the
+    sampled rows, W's everywhere, D within tolerance on the sampled rows."""
+    m = n = k = 8192
+    x, w = workloads.prefill_inputs()
+    qx = fp4.quantize(x.cuda(), fp4.MXFP8, 32)
+    qw = fp4.quantize(w.cuda(), fp4.MXFP4, 32)
+    d = fp4.gemm_mixed(qx, qw, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_status() == fp4.OK
+    rows = _sample(m, 5)
+    qx_o, x_hat = _oracle_rows_1d(host_input(x), rows, fp4.MXFP8, 32)
+    assert np.array_equal(qx.codes.cpu().numpy()[rows], qx_o["codes"])
+    assert np.array_equal(oracle.unswizzle_scales(qx.scales.cpu().numpy(), m, k // 32)[rows], qx_o["scales"])
+    ow = oracle.quantize(host_input(w), fp4.MXFP4, 32)
+    assert np.array_equal(qw.codes.cpu().numpy(), ow["codes"])
+    w_hat = oracle.dequantize(ow["codes"], ow["scales"], ow["g"], fp4.MXFP4)
+    _check_rows(d, rows, x_hat, w_hat, "mixed MXFP8 x MXFP4")
