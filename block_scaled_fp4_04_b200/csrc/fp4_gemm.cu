@@ -228,7 +228,7 @@ constexpr int pipes_per_cta() { return BN <= 32 ? FP4_SMALL_N_PIPES : BN <= 64 ?
 // memory, an E8M0 scale per 32): a stage holds 128 K elements, one scale atom per row-block.
 template <int BN, bool MX, int ACC, bool PAIR = false, bool F8 = false>
 struct Cfg {
-  static_assert(!F8 || (MX && !PAIR), "mixed-format MMAs: E8M0 scales, single-CTA tiles");
+  static_assert(!F8 || MX, "mixed-format MMAs: E8M0 scales");
   static_assert(!PAIR || (BN == 256 && ACC == 1), "CTA pairs run 256 x 256 tiles");
   static constexpr int kP = pipes_per_cta<BN>();
   // Single-pipeline kernels (128/256-wide tiles) add copier warps that move each stage's
@@ -634,7 +634,7 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR, F8>::kThreads, 1)
           if constexpr (PAIR) {
             if (leader) {  // the leader's barriers count the boxes of both CTAs
               mbar_arrive_expect_tx(&sf_landed[stage], 2 * (C::kSFABytes + C::kSFBBytes));
-              mbar_arrive_expect_tx(&full[stage], 2 * (C::kABytes + C::kBBytes));
+              mbar_arrive_expect_tx(&full[stage], 2 * ab_tx);
             }
           } else if constexpr (C::kSepCp) {
             mbar_arrive_expect_tx(&sf_landed[stage], stage_sf_bytes(w, kb));
@@ -719,8 +719,12 @@ __global__ void __launch_bounds__(Cfg<BN, MX, ACC, PAIR, F8>::kThreads, 1)
               const uint32_t sfid = static_cast<uint32_t>(k);
               const uint32_t idesc = mma_idesc_f8(BN, p.f8_fmt & 7u, (p.f8_fmt >> 3) & 7u, sfid, sfid, kMTile);
               const uint32_t accum = (kb > w.kb0 || k > 0) ? 1u : 0u;
-              tc_mma_mxf8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t | (sfid << 30), sfb_t | (sfid << 30),
-                              accum);
+              if constexpr (PAIR)
+                tc_mma_mxf8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t | (sfid << 30),
+                                     sfb_t | (sfid << 30), accum);
+              else
+                tc_mma_mxf8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t | (sfid << 30),
+                                sfb_t | (sfid << 30), accum);
             }
           } else {
           for (int k = 0; k < nk; ++k) {
@@ -1435,18 +1439,29 @@ int launch_gemm_mixed(const GemmProblem& g, int a_fp8, int b_fp8, unsigned* stat
   const int sms = num_sms();
   const int64_t tiles256 = ((g.M + 127) / 128) * ((g.N + 255) / 256);
   const int BN = (g.N >= 256 && tiles256 >= sms) ? 256 : 128;
-  CUtensorMap ta, tb;
+  // 256-wide tiles with at least two 128-row blocks run on CTA pairs, as the FP4 GEMM's do
+  const bool pair = BN == 256 && g.M >= 256;
+  CUtensorMap ta, tb, tsa, tsb;
   const bool ok_a = a_fp8 ? make_tensor_map_u8(&ta, g.A, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M), 128)
                           : encode_map_u4(&ta, g.A, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M), 128);
   const bool ok_b = b_fp8 ? make_tensor_map_u8(&tb, g.B, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N),
-                                               static_cast<uint32_t>(BN))
+                                               static_cast<uint32_t>(pair ? BN / 2 : BN))
                           : encode_map_u4(&tb, g.B, static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N),
-                                          static_cast<uint32_t>(BN));
+                                          static_cast<uint32_t>(pair ? BN / 2 : BN));
   if (!ok_a || !ok_b) {
     *why = "cuTensorMapEncodeTiled failed (alignment or driver)";
     return 1;
   }
   const int64_t atoms_k = g.K / 128;  // one E8M0 per 32 K elements, four per atom row
+  tsa = ta;
+  tsb = ta;
+  // a pair loads a stage's scale atoms (one per 128-row block: 512 bytes, two 256-byte rows)
+  // with tensor copies that complete on the leader's barrier
+  if (pair && (!make_sf_map(&tsa, g.sA, static_cast<uint64_t>((g.M + 127) / 128) * atoms_k * 512, 2) ||
+               !make_sf_map(&tsb, g.sB, static_cast<uint64_t>((g.N + 127) / 128) * atoms_k * 512, 2))) {
+    *why = "cuTensorMapEncodeTiled failed for the scale factors (alignment or driver)";
+    return 1;
+  }
   GemmArgs a{};
   a.sfa = g.sA;
   a.sfb = g.sB;
@@ -1464,14 +1479,15 @@ int launch_gemm_mixed(const GemmProblem& g, int a_fp8, int b_fp8, unsigned* stat
   const int esz = g.out_bf16 ? 2 : 4;
   a.vec_store = ((g.N * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(g.D) & 15) == 0) ? 1 : 0;
   a.mode = kModeTile;
-  a.tiles_m = static_cast<int>((g.M + 127) / 128);
+  a.tiles_m = static_cast<int>((g.M + (pair ? 255 : 127)) / (pair ? 256 : 128));
   a.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
   a.group_m = 16;
   a.total_units = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
   a.status = status;
   a.f8_fmt = (a_fp8 ? kFmtE4M3 : kFmtE2M1) | ((b_fp8 ? kFmtE4M3 : kFmtE2M1) << 3);
-  const cudaError_t e = BN == 256 ? run<256, true, 1, false, true>(ta, tb, ta, tb, a, a.total_units, st)
-                                  : run<128, true, 2, false, true>(ta, tb, ta, tb, a, a.total_units, st);
+  const cudaError_t e = pair        ? run<256, true, 1, true, true>(ta, tb, tsa, tsb, a, a.total_units, st)
+                        : BN == 256 ? run<256, true, 1, false, true>(ta, tb, tsa, tsb, a, a.total_units, st)
+                                    : run<128, true, 2, false, true>(ta, tb, tsa, tsb, a, a.total_units, st);
   if (e != cudaSuccess) {
     *err = e;
     return 2;
