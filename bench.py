@@ -726,9 +726,16 @@ def measure_quantize(args, dev, peaks, cpu: bool) -> dict:
     """The quantize kernels alone (GB/s of algorithmic bytes; NVFP4 reads x twice: the tensor
     amax, then the encode)."""
     import block_scaled_fp4_04_b200 as fp4
+    moe = {}
+
+    def moe_activations():
+        a, _, offsets, _ = workloads.moe_inputs(device="cpu", n=32)
+        moe["offsets"] = offsets
+        return a
+
     cases = [
-        ("moe_quantize", "MoE activations bf16 [16384, 2880] -> MXFP4",
-         lambda: workloads.moe_inputs(device="cpu", n=32)[0], fp4.MXFP4, 32),
+        ("moe_quantize", "MoE activations bf16 [16384, 2880] -> MXFP4, grouped by expert (32 experts, one pass)",
+         moe_activations, fp4.MXFP4, 32),
         ("quantize_train_x", "train X bf16 [16384, 16384] -> NVFP4 (amax + encode)",
          lambda: workloads.train_inputs(16384, device="cpu")[0], fp4.NVFP4, 16),
         ("quantize_decode_w", "decode W fp32 [28672, 8192] -> NVFP4 (amax + encode)",
@@ -764,8 +771,22 @@ def measure_quantize(args, dev, peaks, cpu: bool) -> dict:
             nbytes = 2 * rows * cols * esz + codes + sc
         else:
             nbytes = rows * cols * esz + codes + sc
-        ms, batches, clk = timed_batches(lambda i: fp4.quantize(x, fmt, blk, workspace=ws), max(3, args.steps // 4),
-                                         args.warmup, di, min_s=0.25)
+        run = lambda i: fp4.quantize(x, fmt, blk, workspace=ws)
+        if key == "moe_quantize":
+            # the grouped layout an MoE layer's GEMM reads: one scale byte per block written
+            off = moe["offsets"].to(dev)
+            E = off.numel() - 1
+            gcodes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+            gsc = torch.empty(fp4.fp4_scales_bytes_grouped(rows, E, cols, fmt), dtype=torch.uint8, device=dev)
+            L = fp4.lib()
+            sp = torch.cuda.current_stream().cuda_stream
+            nbytes = rows * cols * esz + codes + rows * (cols // blk)
+
+            def run(i):
+                if L.fp4_quantize_grouped(x.data_ptr(), rows, cols, fp4.BF16, fmt, E, off.data_ptr(),
+                                          gcodes.data_ptr(), gsc.data_ptr(), None, None, None, 0, sp):
+                    raise RuntimeError(fp4.fp4_last_error())
+        ms, batches, clk = timed_batches(run, max(3, args.steps // 4), args.warmup, di, min_s=0.25)
         _check(fp4)
         gbs = nbytes / (ms * 1e-3) / 1e9
         rec = {"case": name, "ms": ms, "GB/s": gbs, "bytes": nbytes,

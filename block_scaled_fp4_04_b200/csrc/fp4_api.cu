@@ -121,6 +121,7 @@ static fp4_status quantize_common(const void* x, int64_t rows, int64_t cols, fp4
   if (!x || !codes || !scales) return fail(FP4_ERR_INVALID_ARG, "null pointer");
   if (rows <= 0 || cols <= 0) return fail(FP4_ERR_INVALID_ARG, "rows and cols must be positive");
   if (cols % 32 != 0) return fail(FP4_ERR_INVALID_ARG, "cols must be a multiple of 32");
+  if (rows > (1ll << 31) - 256) return fail(FP4_ERR_UNSUPPORTED, "rows too large");  // row offsets are int32
   if (in_dtype != FP4_F32 && in_dtype != FP4_BF16) return fail(FP4_ERR_INVALID_ARG, "in_dtype");
   if (fmt != FP4_NVFP4 && fmt != FP4_MXFP4 && fmt != FP4_MXFP8) return fail(FP4_ERR_INVALID_ARG, "fmt");
   if (fmt == FP4_MXFP8) {

@@ -310,7 +310,7 @@ __device__ __forceinline__ uint32_t chunk_absmax_bf16(const uint4& u) {
   return max(w << 16, w & 0xFFFF0000u);
 }
 
-template <typename T, int BLOCK, bool MX, bool HW, int VAR = kQuantPlain>
+template <typename T, int BLOCK, bool MX, bool HW, int VAR = kQuantPlain, bool GROUPED = false>
 __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int EPC = Elem<T>::kPerChunk;
   constexpr int CH = BLOCK * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per block
@@ -320,24 +320,20 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
   static_assert(VAR != kQuantFp8 || (MX && BLOCK == 32), "MXFP8: E4M3 elements in 32-blocks");
   constexpr int RW = VAR == kQuantSR ? BLOCK / 4 : 0;  // 16-byte loads of random words per block
 
-  __shared__ int s_rb[kMaxGroups + 1];
-  __shared__ int s_off[kMaxGroups + 1];
-
+  // grouped: 2 (E + 1) ints, sized at launch; ungrouped launches take no shared memory and
+  // no barrier (a fixed 8 KB table for the largest group count, or the barrier, cost the
+  // streaming loads about 1 us of a 25 us launch)
+  extern __shared__ int s_grp[];
+  int* const s_rb = s_grp;
+  int* const s_off = s_grp + (GROUPED ? p.num_groups + 1 : 0);
   allow_dependents();
   wait_prior_grids();  // g (and x, offsets) may come from the kernels just before
-  const int E = p.offsets ? p.num_groups : 1;
-  if (p.offsets) {
+  const int E = GROUPED ? p.num_groups : 1;
+  int rb_total = static_cast<int>((p.rows + 127) / 128);
+  if constexpr (GROUPED) {
     group_prefix(p.offsets, E, s_rb, s_off);
-  } else {
-    if (threadIdx.x == 0) {
-      s_rb[0] = 0;
-      s_rb[1] = static_cast<int>((p.rows + 127) / 128);
-      s_off[0] = 0;
-      s_off[1] = static_cast<int>(p.rows);
-    }
-    __syncthreads();
+    rb_total = s_rb[E];
   }
-  const int rb_total = s_rb[E];
   float g = 1.0f;
   if constexpr (!MX) g = *p.g;
 
@@ -355,9 +351,11 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       if (tid < 32) reinterpret_cast<uint4*>(atom)[tid] = make_uint4(0, 0, 0, 0);
       continue;
     }
-    // group of this row-block (binary search over the prefix)
+    // group of this row-block (binary search over the prefix).  A tile never spans two
+    // groups: tiles of x's own 128-row blocks, each scale byte sent to its group's atom,
+    // measured 20% slower on 32 groups of ~512 rows.
     int e = 0;
-    if (E > 1) {
+    if (GROUPED && E > 1) {
       int lo = 0, hi = E - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -366,8 +364,8 @@ __global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
       }
       e = lo;
     }
-    const int64_t row_base = s_off[e] + (rb - s_rb[e]) * 128;
-    const int64_t row_end = s_off[e + 1];
+    const int64_t row_base = GROUPED ? s_off[e] + (rb - s_rb[e]) * 128 : rb * 128;
+    const int64_t row_end = GROUPED ? s_off[e + 1] : p.rows;
 
     // this thread's blocks: unit q -> row q / 4 of the tile, block column q % 4
     uint4 u[UPT][CH];
@@ -848,6 +846,12 @@ static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if constexpr (VAR == kQuantPlain) {
+    cfg.dynamicSmemBytes = a.offsets ? 2 * (a.num_groups + 1) * sizeof(int) : 0;
+    if (a.offsets) return cudaLaunchKernelEx(&cfg, quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware, VAR, true>, a);
+  } else {
+    if (a.offsets) return cudaErrorInvalidValue;  // the variants take no groups
+  }
   return cudaLaunchKernelEx(&cfg, quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware, VAR>, a);
 }
 

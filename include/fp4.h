@@ -105,8 +105,8 @@ fp4_status fp4_amax(const void* x_dev, int64_t n, fp4_dtype in_dtype, float* ama
  *              scales fp4_scales_bytes(cols, rows, NVFP4); NULL otherwise.
  *   global_in_dev: NULL -> compute amax and g on the device (two passes over x);
  *              else the caller's g (one pass; e.g. a calibrated scale).
- * Requires cols % 32 == 0, rows >= 1; block 256 also rows % 32 == 0; x, codes and
- * scales 16-byte aligned.  NVFP4 block scale: sb = E4M3_rn_sat((amax_b / 6) / g);
+ * Requires cols % 32 == 0, 1 <= rows <= 2^31 - 256 (else FP4_ERR_UNSUPPORTED); block 256
+ * also rows % 32 == 0; x, codes and scales 16-byte aligned.  NVFP4 block scale: sb = E4M3_rn_sat((amax_b / 6) / g);
  * elements x * (1 / (dec(sb) * g)) in FP32.  MXFP4: sb = E8M0 nearest power of two of
  * amax_b / 6 (a midpoint goes up); elements x * 2^(127 - sb).  MXFP8: sb = E8M0 nearest
  * power of two of amax_b / 448 (the pages fix no rule for MXFP8; 448 is E4M3's largest

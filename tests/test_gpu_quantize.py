@@ -165,6 +165,49 @@ def test_grouped_quantize_layout():
         assert not got[sw.size:].any()   # the rest of the bound is zero pad
 
 
+GROUP_OFFSETS = [
+    # whole 128-row atoms, an empty group, three one-row groups inside one tile, ragged end
+    [0, 128, 256, 257, 257, 300, 301, 302, 303, 430, 640, 700],
+    # 128 one-row groups (all ending in the first tile), then 6- and 5-row groups
+    list(range(0, 129)) + [129 + 5 * k for k in range(1, 40)],
+    # leading empty groups, then one group over eight tiles, ending on a tile boundary
+    [0, 0, 0, 1024],
+    # one group of one row
+    [0, 1],
+]
+
+
+@pytest.mark.parametrize("offsets", GROUP_OFFSETS, ids=["atoms", "one_row_groups", "empty_lead", "one_row"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_grouped_quantize_layout_group_patterns(offsets, dtype):
+    """Groups that begin and end anywhere in a 128-row tile of x: each row's scale byte goes
+    to its group's atom, the lanes past a group's rows and the atoms past the last group's
+    are zero, up to the buffer's bound (pre-filled with a marker)."""
+    offsets = np.array(offsets, np.int32)
+    rows, cols, E = int(offsets[-1]), 320, len(offsets) - 1   # 320: a ragged column tile
+    x = random_input(rows, cols, 5 + E, dtype)
+    off_d = torch.from_numpy(offsets).cuda()
+    dt = fp4.BF16 if dtype == torch.bfloat16 else fp4.F32
+    for fmt in (fp4.MXFP4, fp4.NVFP4):
+        blk = 32 if fmt == fp4.MXFP4 else 16
+        cap = fp4.fp4_scales_bytes_grouped(rows, E, cols, fmt)
+        codes = torch.full((rows, cols // 2), 0xCD, dtype=torch.uint8, device="cuda")
+        scales = torch.full((cap,), 0xAB, dtype=torch.uint8, device="cuda")
+        g = torch.empty(1, dtype=torch.float32, device="cuda")
+        ws = torch.zeros(fp4.fp4_quantize_workspace_size(), dtype=torch.uint8, device="cuda")
+        fp4.fp4_quantize_grouped(x.cuda(), rows, cols, dt, fmt, E, off_d, codes, scales, g, None, ws, ws.numel())
+        torch.cuda.synchronize()
+        assert fp4.fp4_get_status() == fp4.OK
+        oq = oracle_quantize(x, fmt, blk)
+        sw = oracle.swizzle_scales_grouped(oq["scales"], offsets)
+        got = scales.cpu().numpy()
+        assert np.array_equal(codes.cpu().numpy(), oq["codes"])
+        assert np.array_equal(got[:sw.size], sw)
+        assert not got[sw.size:].any()
+        if fmt == fp4.NVFP4:
+            assert np.float32(g.item()).tobytes() == np.float32(oq["g"]).tobytes()
+
+
 def test_dequantize_matches_oracle():
     x = random_input(130, 256, 31)
     for fmt, blk in ((fp4.NVFP4, 16), (fp4.MXFP4, 32)):
