@@ -310,8 +310,15 @@ __device__ __forceinline__ uint32_t chunk_absmax_bf16(const uint4& u) {
   return max(w << 16, w & 0xFFFF0000u);
 }
 
+// BF16 input in 16-blocks (plain and Hadamard) fits five CTAs per SM without spilling; the
+// encode pass is issue-bound, and the extra warps took 4-5% off it (A/B, one B200 session).
+template <typename T, int BLOCK, int VAR>
+constexpr int q1d_min_ctas() {
+  return sizeof(T) == 2 && BLOCK == 16 && VAR != kQuantSR ? 5 : 0;
+}
+
 template <typename T, int BLOCK, bool MX, bool HW, int VAR = kQuantPlain, bool GROUPED = false>
-__global__ void __launch_bounds__(256) quantize_1d_kernel(const Quant1DArgs p) {
+__global__ void __launch_bounds__(256, q1d_min_ctas<T, BLOCK, VAR>()) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int EPC = Elem<T>::kPerChunk;
   constexpr int CH = BLOCK * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per block
   constexpr int UPT = 2;                                        // blocks per thread per tile

@@ -61,6 +61,44 @@ def test_quantize_caller_global_scale():
         assert_quant_equal(gq, oracle_quantize(x, fp4.NVFP4, 16, g_in=np.float32(g)), f"g={g}")
 
 
+def _near_midpoint_maxima(g32: np.float32) -> np.ndarray:
+    """Block maxima a whose quotient (a / 6) / g lands within 24 float steps of each point
+    where the E4M3 code changes: the midpoints between E4M3 values (subnormal ones too),
+    2^-6, and 448 and above (saturation)."""
+    vals = sorted({oracle.e4m3_decode(c) for c in range(1, 127)})
+    marks = [(a + b) / 2 for a, b in zip(vals, vals[1:])] + [2.0 ** -6, 448.0, 464.0, 480.0, 1e4]
+    out = []
+    for m in marks:
+        a0 = np.float32(np.float64(m) * 6.0 * np.float64(g32))
+        if not np.isfinite(a0) or a0 == 0:
+            continue
+        bits = int(a0.view(np.uint32))
+        out.extend(np.array([bits + d for d in range(-24, 25)], np.uint32).view(np.float32))
+    return np.array(out, np.float32)
+
+
+@pytest.mark.parametrize("g", [1.0, 0.37, 3.1e-5, 7.7e4, 2.0 ** -20, 2.0 ** -70, 2.0 ** 70])
+def test_nvfp4_block_scale_near_e4m3_midpoints(g):
+    """Block maxima on both sides of every point where the E4M3 scale code changes, for
+    global scales inside and far outside the usual range: scale bytes and codes equal the
+    oracle's (two FP32 divisions, then E4M3 rounding).  The tensor holds more blocks than
+    the single-launch path for small tensors takes, so the 1-D encode kernel runs."""
+    g32 = np.float32(g)
+    amaxes = _near_midpoint_maxima(g32)
+    rows, cols = 640, 256
+    nb = rows * cols // 16
+    assert nb > 8192 and amaxes.size <= nb
+    rng = np.random.default_rng(12)
+    frac = rng.uniform(-0.999, 0.999, size=(nb, 15)).astype(np.float32)
+    a = np.ones(nb, np.float32)
+    a[:amaxes.size] = amaxes
+    blocks = np.concatenate([a[:, None], (a[:, None] * frac).astype(np.float32)], axis=1)
+    x = torch.from_numpy(np.ascontiguousarray(blocks.reshape(rows, cols)))
+    gq = gpu_quantize(x.cuda(), fp4.NVFP4, 16, g_in=float(g32))
+    torch.cuda.synchronize()
+    assert_quant_equal(gq, oracle_quantize(x, fp4.NVFP4, 16, g_in=g32), f"g={g}")
+
+
 def _golden_blocks():
     path = os.path.join(os.path.dirname(__file__), "golden", "worked_blocks.txt")
     out = []
