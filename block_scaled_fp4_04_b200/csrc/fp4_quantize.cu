@@ -312,13 +312,13 @@ __device__ __forceinline__ uint32_t chunk_absmax_bf16(const uint4& u) {
 
 // BF16 input in 16-blocks (plain and Hadamard) fits five CTAs per SM without spilling; the
 // encode pass is issue-bound, and the extra warps took 4-5% off it (A/B, one B200 session).
-template <typename T, int BLOCK, int VAR>
+template <typename T, int BLOCK, int VAR, bool GROUPED>
 constexpr int q1d_min_ctas() {
-  return sizeof(T) == 2 && BLOCK == 16 && VAR != kQuantSR ? 5 : 0;
+  return sizeof(T) == 2 && BLOCK == 16 && VAR != kQuantSR && !GROUPED ? 5 : 0;
 }
 
 template <typename T, int BLOCK, bool MX, bool HW, int VAR = kQuantPlain, bool GROUPED = false>
-__global__ void __launch_bounds__(256, q1d_min_ctas<T, BLOCK, VAR>()) quantize_1d_kernel(const Quant1DArgs p) {
+__global__ void __launch_bounds__(256, q1d_min_ctas<T, BLOCK, VAR, GROUPED>()) quantize_1d_kernel(const Quant1DArgs p) {
   constexpr int EPC = Elem<T>::kPerChunk;
   constexpr int CH = BLOCK * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per block
   constexpr int UPT = 2;                                        // blocks per thread per tile
@@ -327,19 +327,40 @@ __global__ void __launch_bounds__(256, q1d_min_ctas<T, BLOCK, VAR>()) quantize_1
   static_assert(VAR != kQuantFp8 || (MX && BLOCK == 32), "MXFP8: E4M3 elements in 32-blocks");
   constexpr int RW = VAR == kQuantSR ? BLOCK / 4 : 0;  // 16-byte loads of random words per block
 
-  // grouped: 2 (E + 1) ints, sized at launch; ungrouped launches take no shared memory and
-  // no barrier (a fixed 8 KB table for the largest group count, or the barrier, cost the
-  // streaming loads about 1 us of a 25 us launch)
+  // More than 32 groups: the row-block prefix in shared memory, 2 (E + 1) ints sized at
+  // launch.  Up to 32 groups: every warp forms the prefix in registers (lane e holds group
+  // e), with no shared memory and no barrier.  Ungrouped launches take neither (a fixed 8 KB
+  // table for the largest group count, or a barrier, cost the streaming loads about 1 us of
+  // a 25 us launch).
   extern __shared__ int s_grp[];
   int* const s_rb = s_grp;
   int* const s_off = s_grp + (GROUPED ? p.num_groups + 1 : 0);
   allow_dependents();
   wait_prior_grids();  // g (and x, offsets) may come from the kernels just before
   const int E = GROUPED ? p.num_groups : 1;
+  const int lane = threadIdx.x & 31;
   int rb_total = static_cast<int>((p.rows + 127) / 128);
+  int w_off = 0, w_end = 0, w_rb = 0, w_rbe = 0;  // lane e < E: offsets[e], offsets[e + 1], rb[e], rb[e + 1]
   if constexpr (GROUPED) {
-    group_prefix(p.offsets, E, s_rb, s_off);
-    rb_total = s_rb[E];
+    if (E <= 32) {
+      if (lane < E) {
+        w_off = p.offsets[lane];
+        w_end = p.offsets[lane + 1];
+      }
+      const int cnt = lane < E ? (w_end - w_off + 127) / 128 : 0;
+      int incl = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += t;
+      }
+      w_rb = incl - cnt;
+      w_rbe = incl;
+      rb_total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    } else {
+      group_prefix(p.offsets, E, s_rb, s_off);
+      rb_total = s_rb[E];
+    }
   }
   float g = 1.0f;
   if constexpr (!MX) g = *p.g;
@@ -358,21 +379,29 @@ __global__ void __launch_bounds__(256, q1d_min_ctas<T, BLOCK, VAR>()) quantize_1
       if (tid < 32) reinterpret_cast<uint4*>(atom)[tid] = make_uint4(0, 0, 0, 0);
       continue;
     }
-    // group of this row-block (binary search over the prefix).  A tile never spans two
-    // groups: tiles of x's own 128-row blocks, each scale byte sent to its group's atom,
-    // measured 20% slower on 32 groups of ~512 rows.
-    int e = 0;
-    if (GROUPED && E > 1) {
-      int lo = 0, hi = E - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_rb[mid] <= rb) lo = mid;
-        else hi = mid - 1;
+    // group of this row-block: one ballot over the warp's prefix (<= 32 groups), else a binary
+    // search of the shared table.  A tile never spans two groups: tiles of x's own 128-row
+    // blocks, each scale byte sent to its group's atom, measured 20% slower (32 x ~512 rows).
+    int64_t row_base = rb * 128, row_end = p.rows;
+    if constexpr (GROUPED) {
+      if (E <= 32) {
+        // the one lane (group) whose row-blocks hold rb; none only for malformed offsets
+        const unsigned own = __ballot_sync(0xFFFFFFFFu, lane < E && w_rb <= rb && rb < w_rbe);
+        const int e = own ? __ffs(own) - 1 : 0;
+        row_base = __shfl_sync(0xFFFFFFFFu, w_off, e) + (rb - __shfl_sync(0xFFFFFFFFu, w_rb, e)) * 128;
+        row_end = own ? __shfl_sync(0xFFFFFFFFu, w_end, e) : row_base;
+      } else {
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (s_rb[mid] <= rb) lo = mid;
+          else hi = mid - 1;
+        }
+        row_base = s_off[lo] + (rb - s_rb[lo]) * 128;
+        row_end = s_off[lo + 1];
       }
-      e = lo;
+      if (row_end > p.rows) row_end = p.rows;  // offsets past the tensor read nothing
     }
-    const int64_t row_base = GROUPED ? s_off[e] + (rb - s_rb[e]) * 128 : rb * 128;
-    const int64_t row_end = GROUPED ? s_off[e + 1] : p.rows;
 
     // this thread's blocks: unit q -> row q / 4 of the tile, block column q % 4
     uint4 u[UPT][CH];
@@ -383,7 +412,7 @@ __global__ void __launch_bounds__(256, q1d_min_ctas<T, BLOCK, VAR>()) quantize_1
       const int q = tid + 256 * i;
       const int64_t r = row_base + (q >> 2);
       const int64_t bcol = ct * 4 + (q & 3);
-      ok[i] = r < row_end && bcol < nbc;
+      ok[i] = (!GROUPED || r >= 0) && r < row_end && bcol < nbc;
       const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) +
                                                         (r * p.cols + bcol * BLOCK) * static_cast<int64_t>(sizeof(T)));
 #pragma unroll
@@ -854,7 +883,7 @@ static cudaError_t launch_q1d_t(const Quant1DArgs& a, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if constexpr (VAR == kQuantPlain) {
-    cfg.dynamicSmemBytes = a.offsets ? 2 * (a.num_groups + 1) * sizeof(int) : 0;
+    cfg.dynamicSmemBytes = a.offsets && a.num_groups > 32 ? 2 * (a.num_groups + 1) * sizeof(int) : 0;
     if (a.offsets) return cudaLaunchKernelEx(&cfg, quantize_1d_kernel<T, BLOCK, MX, kE2M1Hardware, VAR, true>, a);
   } else {
     if (a.offsets) return cudaErrorInvalidValue;  // the variants take no groups
