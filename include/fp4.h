@@ -106,11 +106,12 @@ fp4_status fp4_amax(const void* x_dev, int64_t n, fp4_dtype in_dtype, float* ama
  *   global_in_dev: NULL -> compute amax and g on the device (two passes over x);
  *              else the caller's g (one pass; e.g. a calibrated scale).
  * Requires cols % 32 == 0, 1 <= rows <= 2^31 - 256 (else FP4_ERR_UNSUPPORTED); block 256
- * also rows % 32 == 0; x, codes and scales 16-byte aligned.  NVFP4 block scale: sb = E4M3_rn_sat((amax_b / 6) / g);
- * elements x * (1 / (dec(sb) * g)) in FP32.  MXFP4: sb = E8M0 nearest power of two of
- * amax_b / 6 (a midpoint goes up); elements x * 2^(127 - sb).  MXFP8: sb = E8M0 nearest
- * power of two of amax_b / 448 (the pages fix no rule for MXFP8; 448 is E4M3's largest
- * value as 6 is E2M1's); elements E4M3_rn_sat(x * 2^(127 - sb)), sign in bit 7. */
+ * also rows % 32 == 0; x, codes and scales 16-byte aligned.  NVFP4 block scale:
+ * sb = E4M3_rn_sat((amax_b / 6) / g); elements x * (1 / (dec(sb) * g)) in FP32.  MXFP4:
+ * sb = E8M0 nearest power of two of amax_b / 6 (a midpoint goes up); elements
+ * x * 2^(127 - sb).  MXFP8: sb = E8M0 nearest power of two of amax_b / 448 (the sources
+ * cited above fix no rule for MXFP8; 448 is E4M3's largest value as 6 is E2M1's); elements
+ * E4M3_rn_sat(x * 2^(127 - sb)), sign in bit 7. */
 fp4_status fp4_quantize(const void* x_dev, int64_t rows, int64_t cols, fp4_dtype in_dtype,
                         fp4_fmt fmt, int block, uint8_t* codes_out_dev, uint8_t* scales_out_dev,
                         float* global_out_dev, uint8_t* codesT_out_dev, uint8_t* scalesT_out_dev,
@@ -280,8 +281,8 @@ fp4_status fp4_gemm_bf16a(const void* X_dev, const uint8_t* B_dev, const uint8_t
                           uint8_t* Xcodes_dev, uint8_t* Xscales_dev, float* gX_dev,
                           void* workspace_dev, size_t workspace_bytes, unsigned flags, void* stream);
 
-/* fp4_gemm for callers that cannot allocate device memory.  The pages have no
- * counterpart to this entry point.  Some hosts own every byte of device memory and give
+/* fp4_gemm for callers that cannot allocate device memory.  The sources cited above
+ * have no counterpart to this entry point.  Some hosts own every byte of device memory and give
  * this library no allocator: plugin runtimes and embedded inference engines that carve
  * one arena out of the GPU at start-up and treat any later cudaMalloc as a failure.
  * Arguments as fp4_gemm minus the workspace.  The split-K scratch that decode-sized

@@ -366,8 +366,8 @@ def epilogue(d: np.ndarray, bias=None, act: str = "none") -> np.ndarray:
     result is multiplied by the scale factors, the bias is added, the activation is
     applied, then it is converted to the output format; 4.2: C = (A.B)(sA.sB) + bias).
     ``d`` is the scaled product (``gemm_reference`` of the dequantized operands);
-    ``bias`` [N] is added to every row; ``act`` is "none" or "relu" (the pages name no
-    activation; ReLU is the plainest).  FP64."""
+    ``bias`` [N] is added to every row; ``act`` is "none" or "relu" (the cited sources
+    name no activation; ReLU is the plainest).  FP64."""
     out = np.asarray(d, dtype=np.float64)
     if bias is not None:
         out = out + np.asarray(bias, dtype=np.float64)[None, :]
